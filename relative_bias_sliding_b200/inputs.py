@@ -1,0 +1,173 @@
+"""Seeded synthetic inputs for the Inkling attention layer.
+
+This module holds no arithmetic of the method: it only draws random tensors
+with fixed seeds, shapes and distributions, in a fixed order, so that the CUDA
+path and the CPU oracle are fed the same arrays.  Distributions follow the
+workloads the layer is measured on: bf16 queries/keys/values N(0, 1), sconv
+taps fp32 N(0, 0.5) (0.5 is the standard deviation), bias tables fp32
+N(0, sigma), paged caches of 128-token blocks placed by a random permutation
+of the block pool.
+
+Draw order (one ``torch.Generator`` per workload, seeded with its seed):
+prefill  q, k_raw, v_raw, w_k, w_v, bias
+decode   q, k_new, v_new, w_k, w_v, bias, k_state, v_state, seq_lens,
+         block permutation, k_cache, v_cache
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, replace
+
+import torch
+
+BLOCK = 128  # tokens per paged-KV block
+
+
+@dataclass(frozen=True)
+class PrefillSpec:
+    name: str
+    B: int
+    T: int
+    Hq: int
+    Hkv: int
+    d: int
+    window: int      # 0 = full causal
+    D_max: int
+    bias_std: float
+    seed: int
+
+    @property
+    def allowed_pairs(self) -> int:
+        """(i, j) pairs inside the causal band / window, per (batch, head)."""
+        T, W = self.T, self.window
+        if W <= 0 or W >= T:
+            return T * (T + 1) // 2
+        return W * (W + 1) // 2 + (T - W) * W
+
+    @property
+    def flops(self) -> int:
+        """Algorithmic FLOPs: 2 contractions of length d per allowed pair."""
+        return 4 * self.d * self.Hq * self.B * self.allowed_pairs
+
+
+@dataclass(frozen=True)
+class DecodeSpec:
+    name: str
+    S: int
+    L_min: int
+    L_max: int       # lengths drawn uniformly in [L_min, L_max]; equal = fixed
+    Hq: int
+    Hkv: int
+    d: int
+    window: int
+    D_max: int
+    bias_std: float
+    seed: int
+    n_new: int = 1
+
+
+WORKLOADS = {
+    # tiny full-causal prefill, small enough for the oracle on every row
+    "prefill_tiny_b1_t256": PrefillSpec("prefill_tiny_b1_t256", 1, 256, 8, 1, 128, 0, 256,
+                                        1.0, 0),
+    # sliding-window prefill, window 4096
+    "prefill_swa_b4_t8192": PrefillSpec("prefill_swa_b4_t8192", 4, 8192, 64, 8, 128, 4096,
+                                        4096, 1.0, 1),
+    # full-attention prefill, 32k tokens
+    "prefill_full_b1_t32768": PrefillSpec("prefill_full_b1_t32768", 1, 32768, 64, 8, 128, 0,
+                                          32768, 0.5, 2),
+    # sliding-window decode over 64 sequences of mixed length
+    "decode_swa_s64": DecodeSpec("decode_swa_s64", 64, 1024, 32768, 64, 8, 128, 4096, 4096,
+                                 1.0, 3),
+    # 1M-token full-attention decode, batch 1 and batch 8
+    "decode_full_1m_b1": DecodeSpec("decode_full_1m_b1", 1, 1 << 20, 1 << 20, 64, 8, 128, 0,
+                                    1 << 20, 0.5, 4),
+    "decode_full_1m_b8": DecodeSpec("decode_full_1m_b8", 8, 1 << 20, 1 << 20, 64, 8, 128, 0,
+                                    1 << 20, 0.5, 4),
+}
+
+
+def scaled(spec, **kw):
+    """Same workload with some sizes replaced (for small parity cases)."""
+    return replace(spec, **kw)
+
+
+def _normal_bf16(gen, shape, device, std=1.0, chunk=1 << 28):
+    """bf16 N(0, std) drawn in fp32 chunks (bounds the fp32 temporary)."""
+    out = torch.empty(shape, dtype=torch.bfloat16, device=device)
+    flat = out.view(-1)
+    n = flat.numel()
+    for s in range(0, n, chunk):
+        e = min(n, s + chunk)
+        tmp = torch.randn(e - s, generator=gen, device=device, dtype=torch.float32)
+        if std != 1.0:
+            tmp.mul_(std)
+        flat[s:e].copy_(tmp)
+    return out
+
+
+def _generator(device, seed):
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def make_prefill(spec: PrefillSpec, device="cpu"):
+    g = _generator(device, spec.seed)
+    B, T, Hq, Hkv, d = spec.B, spec.T, spec.Hq, spec.Hkv, spec.d
+    C = Hkv * d
+    q = _normal_bf16(g, (B, T, Hq, d), device)
+    k_raw = _normal_bf16(g, (B, T, Hkv, d), device)
+    v_raw = _normal_bf16(g, (B, T, Hkv, d), device)
+    w_k = torch.randn((C, 4), generator=g, device=device, dtype=torch.float32) * 0.5
+    w_v = torch.randn((C, 4), generator=g, device=device, dtype=torch.float32) * 0.5
+    bias = torch.randn((Hq, spec.D_max + 1), generator=g, device=device,
+                       dtype=torch.float32) * spec.bias_std
+    return dict(q=q, k_raw=k_raw, v_raw=v_raw, w_k=w_k, w_v=w_v, bias=bias)
+
+
+def make_decode(spec: DecodeSpec, device="cpu", extra_blocks: int = 0):
+    """Decode step inputs.  ``seq_lens`` already count the n_new tokens that the
+    sconv append writes; the cache holds N(0, 1) post-sconv rows for every
+    allocated slot (the append overwrites the new tokens' slots)."""
+    g = _generator(device, spec.seed)
+    S, Hq, Hkv, d, n_new = spec.S, spec.Hq, spec.Hkv, spec.d, spec.n_new
+    C = Hkv * d
+    q = _normal_bf16(g, (S, Hq, d), device)
+    k_new = _normal_bf16(g, (S, n_new, Hkv, d), device)
+    v_new = _normal_bf16(g, (S, n_new, Hkv, d), device)
+    w_k = torch.randn((C, 4), generator=g, device=device, dtype=torch.float32) * 0.5
+    w_v = torch.randn((C, 4), generator=g, device=device, dtype=torch.float32) * 0.5
+    bias = torch.randn((Hq, spec.D_max + 1), generator=g, device=device,
+                       dtype=torch.float32) * spec.bias_std
+    k_state = _normal_bf16(g, (S, 3, C), device)
+    v_state = _normal_bf16(g, (S, 3, C), device)
+    if spec.L_min == spec.L_max:
+        seq_lens = torch.full((S,), spec.L_min, dtype=torch.int32, device=device)
+    else:
+        seq_lens = torch.randint(spec.L_min, spec.L_max + 1, (S,), generator=g,
+                                 device=device, dtype=torch.int64).to(torch.int32)
+    blocks_per_seq = (seq_lens.to(torch.int64) + BLOCK - 1) // BLOCK
+    max_blocks = int(blocks_per_seq.max().item())
+    total = int(blocks_per_seq.sum().item()) + extra_blocks
+    perm = torch.randperm(total, generator=g, device=device).to(torch.int32)
+    block_table = torch.zeros((S, max_blocks), dtype=torch.int32, device=device)
+    off = 0
+    for s in range(S):
+        nb = int(blocks_per_seq[s].item())
+        block_table[s, :nb] = perm[off:off + nb]
+        off += nb
+    k_cache = _normal_bf16(g, (total, Hkv, BLOCK, d), device)
+    v_cache = _normal_bf16(g, (total, Hkv, BLOCK, d), device)
+    return dict(q=q, k_new=k_new, v_new=v_new, w_k=w_k, w_v=w_v, bias=bias,
+                k_state=k_state, v_state=v_state, seq_lens=seq_lens,
+                block_table=block_table, k_cache=k_cache, v_cache=v_cache)
+
+
+def kv_bytes_read(spec: DecodeSpec, seq_lens) -> int:
+    """Post-sconv K+V bytes inside each sequence's window or context."""
+    W = spec.window
+    tot = 0
+    for L in seq_lens.tolist():
+        n = min(L, W) if W > 0 else L
+        tot += n
+    return tot * spec.Hkv * spec.d * 2 * 2
