@@ -1,0 +1,537 @@
+#!/usr/bin/env python3
+"""Benchmark of the Inkling decoder attention layer on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+  * prefill: the sliding-window prefill workload (B=4, T=8192, Hq=64, Hkv=8,
+    d=128, window 4096) through inkling_attn_prefill (sconv fused);
+  * decode: the sliding-window decode workload (64 sequences, lengths uniform
+    in [1024, 32768], window 4096, paged 128-token blocks) through
+    inkling_sconv_kv + inkling_attn_decode.
+The headline ``value`` is prefill TFLOP/s (allowed (i, j) pairs x 4 d Hq B);
+the decode step is reported beside it in KV GB/s (post-sconv K+V bytes inside
+each window).  ``--workload`` picks any single workload instead.
+
+Launch: ``python bench.py --gpus N --steps K --warmup W`` (N > 1 under
+torch.distributed.run: every rank runs the same workload on its own GPU, no
+data-path collective, weak scaling; times are max over ranks).
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
+workload on the host cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "prefill TFLOP/s and decode KV GB/s on 1 B200, as % of BF16/HBM roofline"
+DEFAULT_PREFILL = "prefill_swa_b4_t8192"
+DEFAULT_DECODE = "decode_swa_s64"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------ distributed --
+
+def dist_env():
+    """(rank, world, local_rank) from the torch.distributed.run environment."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def init_dist(world, backend):
+    import datetime
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist if world > 1 else None
+
+
+def barrier(dist, device=None):
+    if dist is not None:
+        if device is not None:
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(dist, values, device="cpu"):
+    """Element-wise max of a list of floats over all ranks (timing only)."""
+    import torch
+    if dist is None:
+        return list(values)
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+# ----------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.fh,
+                stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ peaks --
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------- GPU workload --
+
+class PrefillStep:
+    def __init__(self, spec, device):
+        import torch
+        from relative_bias_sliding_b200.inputs import make_prefill
+        self.spec = spec
+        self.t = make_prefill(spec, device=device)
+        self.out = torch.empty_like(self.t["q"])
+        self.flops = spec.flops
+
+    def run(self, stream=None):
+        import relative_bias_sliding_b200 as ink
+        t = self.t
+        ink.attn_prefill(t["q"], t["k_raw"], t["v_raw"], t["w_k"], t["w_v"], t["bias"],
+                         window=self.spec.window, out=self.out, stream=stream)
+
+    launches = 1
+
+
+class DecodeStep:
+    def __init__(self, spec, device):
+        import torch
+        import relative_bias_sliding_b200 as ink
+        from relative_bias_sliding_b200.inputs import make_decode, kv_bytes_read
+        self.spec = spec
+        self.t = make_decode(spec, device=device)
+        t = self.t
+        self.out = torch.empty_like(t["q"])
+        self.splits = ink.decode_num_splits(t["q"], t["k_cache"], t["v_cache"],
+                                            t["block_table"], t["seq_lens"], t["bias"],
+                                            window=spec.window)
+        nbytes = max(16, ink.decode_workspace_bytes(spec.S, spec.Hq, self.splits))
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.kv_bytes = kv_bytes_read(spec, t["seq_lens"].cpu())
+        self.launches = 2 + (1 if self.splits > 1 else 0)
+
+    def run_append(self, stream=None):
+        import relative_bias_sliding_b200 as ink
+        t = self.t
+        ink.sconv_kv(t["k_new"], t["v_new"], t["w_k"], t["w_v"], t["k_state"], t["v_state"],
+                     t["k_cache"], t["v_cache"], t["block_table"], t["seq_lens"], stream=stream)
+
+    def run_attn(self, stream=None):
+        import relative_bias_sliding_b200 as ink
+        t = self.t
+        ink.attn_decode(t["q"], t["k_cache"], t["v_cache"], t["block_table"], t["seq_lens"],
+                        t["bias"], window=self.spec.window, out=self.out, workspace=self.ws,
+                        num_splits=self.splits, stream=stream)
+
+    def run(self, stream=None):
+        self.run_append(stream)
+        self.run_attn(stream)
+
+
+def timed_loop(steps, fns, stream):
+    """Run ``steps`` iterations of the callables in order on ``stream``; return
+    per-callable mean milliseconds (CUDA events recorded on that stream)."""
+    import torch
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in fns] for _ in range(steps)]
+    for k in range(steps):
+        for (a, b), fn in zip(evs[k], fns):
+            a.record(stream)
+            fn(stream)
+            b.record(stream)
+    stream.synchronize()
+    return [sum(evs[k][i][0].elapsed_time(evs[k][i][1]) for k in range(steps)) / steps
+            for i in range(len(fns))]
+
+
+def e2e_prefill(step, steps, stream):
+    """Same prefill through the public API with host buffers: pinned host ->
+    device copies of the step's inputs, the call, and the output read back."""
+    import torch
+    t = step.t
+    host = {k: t[k].cpu().pin_memory() for k in ("q", "k_raw", "v_raw")}
+    out_h = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    dev = {k: torch.empty_like(t[k]) for k in host}
+    import relative_bias_sliding_b200 as ink
+
+    def once():
+        for k in host:
+            dev[k].copy_(host[k], non_blocking=True)
+        ink.attn_prefill(dev["q"], dev["k_raw"], dev["v_raw"], t["w_k"], t["w_v"], t["bias"],
+                         window=step.spec.window, out=step.out, stream=stream)
+        out_h.copy_(step.out, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        once()
+        stream.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            once()
+        b.record(stream)
+        stream.synchronize()
+    ms = a.elapsed_time(b) / steps
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    return ms, h2d, out_h.numel() * out_h.element_size()
+
+
+def e2e_decode(step, steps, stream):
+    """Decode step through the public API with host buffers for the per-step
+    inputs (queries, new raw keys/values, lengths, block table); the caches
+    and sconv states stay resident as the layer's state."""
+    import torch
+    t = step.t
+    names = ("q", "k_new", "v_new", "seq_lens", "block_table")
+    host = {k: t[k].cpu().pin_memory() for k in names}
+    out_h = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    dev = {k: torch.empty_like(t[k]) for k in names}
+    import relative_bias_sliding_b200 as ink
+
+    def once():
+        for k in names:
+            dev[k].copy_(host[k], non_blocking=True)
+        ink.sconv_kv(dev["k_new"], dev["v_new"], t["w_k"], t["w_v"], t["k_state"], t["v_state"],
+                     t["k_cache"], t["v_cache"], dev["block_table"], dev["seq_lens"],
+                     stream=stream)
+        ink.attn_decode(dev["q"], t["k_cache"], t["v_cache"], dev["block_table"],
+                        dev["seq_lens"], t["bias"], window=step.spec.window, out=step.out,
+                        workspace=step.ws, num_splits=step.splits, stream=stream)
+        out_h.copy_(step.out, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        once()
+        stream.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            once()
+        b.record(stream)
+        stream.synchronize()
+    ms = a.elapsed_time(b) / steps
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    return ms, h2d, out_h.numel() * out_h.element_size()
+
+
+# ------------------------------------------------------------ CPU oracle --
+
+def oracle_prefill_sample(spec, seconds, seed=0):
+    """Time the oracle on a bounded row sample of a prefill workload; returns
+    (TFLOP/s, description, threads)."""
+    import numpy as np
+    import torch
+    import oracle
+    from relative_bias_sliding_b200.inputs import make_prefill
+    t = make_prefill(spec, device="cpu")
+    u = lambda x: x.contiguous().view(torch.int16).numpy().view(np.uint16)
+    rng = np.random.default_rng(seed)
+    W, T = spec.window, spec.T
+    per_row = lambda i: (min(i + 1, W) if W > 0 else i + 1)
+    # calibrate on a small batch, then size the sample to about `seconds`
+    n = 64
+    total_rows, total_flops, total_t = 0, 0, 0.0
+    while True:
+        b = rng.integers(0, spec.B, n)
+        h = rng.integers(0, spec.Hq, n)
+        i = rng.integers(0, T, n)
+        rows = np.stack([b, h, i], 1).astype(np.int32)
+        t0 = time.perf_counter()
+        oracle.prefill_rows(u(t["q"]), u(t["k_raw"]), u(t["v_raw"]), t["w_k"].numpy(),
+                            t["w_v"].numpy(), t["bias"].numpy(), W, spec.D_max, rows)
+        dt = time.perf_counter() - t0
+        total_t += dt
+        total_rows += n
+        total_flops += sum(4 * spec.d * per_row(int(x)) for x in i)
+        if total_t >= seconds:
+            break
+        n = int(min(1 << 16, max(n * 2, n * (seconds - total_t) / max(dt, 1e-3))))
+    desc = (f"{total_rows} random query rows of {spec.name} (sconv of all keys/values "
+            f"included in every call), {total_t:.1f} s")
+    return total_flops / total_t / 1e12, desc, oracle.num_threads()
+
+
+def oracle_decode_sample(spec, seconds, seed=0):
+    """Time the oracle's decode step (sconv append + attention) on whole
+    sequences of a decode workload; returns (KV GB/s, description, threads)."""
+    import numpy as np
+    import torch
+    import oracle
+    from relative_bias_sliding_b200.inputs import make_decode, scaled
+    sub = scaled(spec, S=min(spec.S, 8))
+    t = make_decode(sub, device="cpu")
+    u = lambda x: x.contiguous().view(torch.int16).numpy().view(np.uint16)
+    kc, vc = u(t["k_cache"]).copy(), u(t["v_cache"]).copy()
+    ks, vs = u(t["k_state"]).copy(), u(t["v_state"]).copy()
+    bt, sl = t["block_table"].numpy(), t["seq_lens"].numpy()
+    W = sub.window
+    done_bytes, total_t, nseq = 0, 0.0, 0
+    for s in range(sub.S):
+        pairs = np.array([[s, h] for h in range(sub.Hq)], np.int32)
+        t0 = time.perf_counter()
+        oracle.sconv_append(u(t["k_new"])[s:s + 1], ks[s:s + 1], t["w_k"].numpy(), kc,
+                            bt[s:s + 1], sl[s:s + 1])
+        oracle.sconv_append(u(t["v_new"])[s:s + 1], vs[s:s + 1], t["w_v"].numpy(), vc,
+                            bt[s:s + 1], sl[s:s + 1])
+        oracle.decode_rows(u(t["q"]), kc, vc, bt, sl, t["bias"].numpy(), W, sub.D_max, pairs)
+        total_t += time.perf_counter() - t0
+        L = int(sl[s])
+        done_bytes += (min(L, W) if W > 0 else L) * sub.Hkv * sub.d * 4
+        nseq += 1
+        if total_t >= seconds:
+            break
+    desc = f"{nseq} whole sequences of {spec.name} (all {sub.Hq} heads each), {total_t:.1f} s"
+    return done_bytes / total_t / 1e9, desc, oracle.num_threads()
+
+
+# ------------------------------------------------------------------ main --
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=None,
+                    help="a single workload name from relative_bias_sliding_b200.inputs.WORKLOADS")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def run_reference(args):
+    from relative_bias_sliding_b200.inputs import WORKLOADS, PrefillSpec
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    name = args.workload or DEFAULT_PREFILL
+    spec = WORKLOADS[name]
+    vals = []
+    descs = []
+    per_step = max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    for k in range(args.warmup + args.steps):
+        if isinstance(spec, PrefillSpec):
+            v, desc, thr = oracle_prefill_sample(spec, per_step, seed=k)
+            unit = "TFLOP/s"
+        else:
+            v, desc, thr = oracle_decode_sample(spec, per_step, seed=k)
+            unit = "GB/s"
+        if k >= args.warmup:
+            vals.append(v)
+            descs.append(desc)
+    value = statistics.mean(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": unit,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": name},
+            "cpu_baseline": {"value": value, "unit": unit, "cores": thr, "kind": "oracle",
+                             "sample": descs[0]},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    import torch
+    import relative_bias_sliding_b200 as ink
+    from relative_bias_sliding_b200.inputs import WORKLOADS, PrefillSpec
+
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    ink.load_library()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    if args.workload:
+        spec = WORKLOADS[args.workload]
+        pre = PrefillStep(spec, device) if isinstance(spec, PrefillSpec) else None
+        dec = None if pre else DecodeStep(spec, device)
+    else:
+        pre = PrefillStep(WORKLOADS[DEFAULT_PREFILL], device)
+        dec = DecodeStep(WORKLOADS[DEFAULT_DECODE], device)
+    stream = torch.cuda.Stream(device)
+    fns = []
+    if pre:
+        fns.append(pre.run)
+    if dec:
+        fns += [dec.run_append, dec.run_attn]
+
+    for _ in range(args.warmup):
+        for f in fns:
+            f(stream)
+    stream.synchronize()
+    barrier(dist, device)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        barrier(dist, device)
+        torch.cuda.synchronize()
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        per_fn = timed_loop(args.steps, fns, stream)
+        t_end.record(stream)
+        stream.synchronize()
+        torch.cuda.synchronize()
+        barrier(dist, device)
+    step_ms = t_start.elapsed_time(t_end) / args.steps
+    per_fn = max_over_ranks(dist, per_fn, device)
+    step_ms = max_over_ranks(dist, [step_ms], device)[0]
+
+    e2e = None
+    if not args.no_e2e:
+        e2e_parts = []
+        if pre:
+            e2e_parts.append(("pre",) + e2e_prefill(pre, max(3, args.steps // 4), stream))
+        if dec:
+            e2e_parts.append(("dec",) + e2e_decode(dec, max(3, args.steps // 4), stream))
+        e2e = e2e_parts
+
+    peaks, peak_src = load_peaks()
+    line = {"metric": METRIC, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "gpu_launches": args.steps * sum(x.launches for x in (pre, dec) if x) * 1}
+    i = 0
+    if pre:
+        pre_ms = per_fn[0]
+        i = 1
+        tflops = pre.flops / (pre_ms * 1e-3) / 1e12 * world
+        peak = peaks["bf16_tflops_sustained"]
+        line.update({"value": tflops, "unit": "TFLOP/s"})
+        line["roofline"] = {"bound": "tensor", "kernel": "attn_prefill_kernel",
+                            "achieved": tflops / world, "peak": peak, "unit": "TFLOP/s",
+                            "frac": tflops / world / peak, "traffic": None,
+                            "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed "
+                                           f"inside a long step loop)"}
+    if dec:
+        app_ms, attn_ms = per_fn[i], per_fn[i + 1]
+        gbs = dec.kv_bytes / ((app_ms + attn_ms) * 1e-3) / 1e9
+        kern_gbs = dec.kv_bytes / (attn_ms * 1e-3) / 1e9
+        dec_obj = {"workload": dec.spec.name, "value": gbs * world, "unit": "GB/s",
+                   "ms_per_step": app_ms + attn_ms, "sconv_append_ms": app_ms,
+                   "attn_decode_ms": attn_ms, "num_splits": dec.splits,
+                   "kv_bytes_per_step": dec.kv_bytes,
+                   "roofline": {"bound": "hbm", "kernel": "decode_split_kernel + combine",
+                                "achieved": kern_gbs, "peak": peaks["hbm_gbs"],
+                                "unit": "GB/s", "frac": kern_gbs / peaks["hbm_gbs"],
+                                "traffic": None, "peak_source": f"{peak_src} hbm_gbs"}}
+        if pre:
+            line["decode"] = dec_obj
+        else:
+            line.update({"value": dec_obj["value"], "unit": "GB/s",
+                         "roofline": dec_obj["roofline"]})
+            line["decode"] = {k: v for k, v in dec_obj.items() if k != "roofline"}
+    line["config"] = {"workload": (pre.spec.name if pre else "") +
+                      (" + " if pre and dec else "") + (dec.spec.name if dec else ""),
+                      "parallelism": f"replica per GPU x{world}",
+                      "l2": "inputs larger than L2 (prefill q 512 MiB; decode KV 4.4 GB)"}
+    if e2e:
+        parts = {p[0]: p[1:] for p in e2e}
+        if pre:
+            ms, h2d, d2h = parts["pre"]
+            line["e2e"] = {"value": pre.flops / (ms * 1e-3) / 1e12 * world, "unit": "TFLOP/s",
+                           "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            if dec:
+                ms2, h2d2, d2h2 = parts["dec"]
+                line["e2e"]["decode"] = {"value": dec.kv_bytes / (ms2 * 1e-3) / 1e9 * world,
+                                         "unit": "GB/s", "ms_per_step": ms2,
+                                         "h2d_bytes_per_step": h2d2, "d2h_bytes_per_step": d2h2}
+        else:
+            ms2, h2d2, d2h2 = parts["dec"]
+            line["e2e"] = {"value": dec.kv_bytes / (ms2 * 1e-3) / 1e9 * world, "unit": "GB/s",
+                           "ms_per_step": ms2, "h2d_bytes_per_step": h2d2,
+                           "d2h_bytes_per_step": d2h2}
+    line["clocks"] = clocks.summary()
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        if pre:
+            v, desc, thr = oracle_prefill_sample(pre.spec, args.cpu_seconds)
+            line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": thr,
+                                    "kind": "oracle", "sample": desc}
+        else:
+            v, desc, thr = oracle_decode_sample(dec.spec, args.cpu_seconds)
+            line["cpu_baseline"] = {"value": v, "unit": "GB/s", "cores": thr,
+                                    "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,193 @@
+/*
+ * inkling.h — C ABI of the Inkling decoder attention layer for NVIDIA B200
+ * (sm_100a).
+ *
+ * The layer (vLLM Recipes page "thinkingmachines/Inkling", section Overview,
+ * bullets "Attention" and "Short convolution"):
+ *   1. a causal, depthwise, window-4 short convolution (sconv) over the key
+ *      and value channels:  y[t,c] = sum_{k=0..3} w[c,k] * x[t-k,c], tap 0 =
+ *      current token, rounded once to bf16 (round to nearest even);
+ *   2. grouped-query attention at head size 128 in which RoPE is replaced by
+ *      a learned relative-position term added to the pre-softmax logits:
+ *        s[i,j] = (q_i . k_j) / sqrt(128) + bias[h, min(i-j, D_max)]
+ *      with query head h reading kv head h / (Hq/Hkv);
+ *   3. a sliding-window mask (j allowed iff 0 <= i-j < window) or full causal
+ *      mask (window = 0); the pages split the 66 layers into 55 sliding-window
+ *      and 11 full-attention ones.
+ * The sconv state is kept like the KV cache of a sliding-window layer (same
+ * Overview bullet); the paged KV cache uses 128-token blocks (the
+ * `--block-size 128` launch option in section Client Usage of the same page).
+ *
+ * Conventions shared by every entry point
+ *  - bf16 tensors are passed as `const void*` / `void*` (IEEE bfloat16 bits);
+ *    layouts are row-major, last index contiguous.
+ *  - Every pointer named "device" must point to device memory of the current
+ *    CUDA device and be 16-byte aligned.  The caller owns all memory; the
+ *    library allocates nothing and keeps no state except a per-thread error
+ *    message.
+ *  - Calls are asynchronous on `stream` (NULL = legacy default stream) and
+ *    never synchronise.  Kernel faults surface at the caller's next
+ *    synchronisation, as with any CUDA launch.
+ *  - On invalid arguments a call returns INKLING_ERR_INVALID (or
+ *    INKLING_ERR_UNSUPPORTED for shapes outside what the kernels implement)
+ *    and launches nothing; inkling_last_error() describes why.  A failed
+ *    launch returns INKLING_ERR_CUDA.  No C++ exception crosses this ABI.
+ *  - `status` (optional, nullable, device int32): kernels OR error bits into it
+ *    (INKLING_STATUS_* below) instead of trapping; the caller zeroes it and
+ *    reads it after synchronising.
+ */
+#ifndef INKLING_H
+#define INKLING_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *inkling_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    INKLING_OK = 0,
+    INKLING_ERR_INVALID = 1,     /* bad pointer / shape / size; nothing launched */
+    INKLING_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. head_dim != 128) */
+    INKLING_ERR_CUDA = 3         /* a CUDA runtime / driver call failed */
+} inkling_status;
+
+/* bits a kernel may OR into the optional device status word */
+#define INKLING_STATUS_TIMEOUT 1      /* a bounded wait inside a kernel gave up */
+#define INKLING_STATUS_BAD_BLOCK 2    /* a block-table entry was outside [0, num_blocks) */
+#define INKLING_STATUS_BAD_LENGTH 4   /* a sequence length was outside [1, max_blocks*128] */
+
+/* Head dimension and paged-cache block size the kernels are built for. */
+#define INKLING_HEAD_DIM 128
+#define INKLING_BLOCK_SIZE 128
+
+/* Message for the last failed call on this host thread ("" if none). */
+const char *inkling_last_error(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int inkling_version(void);
+
+/* --------------------------------------------------------------------------
+ * inkling_sconv_kv — decode-side sconv append (Overview, "Short convolution":
+ * the sconv on keys and values, with its state kept as a sliding-window
+ * cache).
+ *
+ * For every sequence s and each of its n_new new tokens (positions
+ * L-n_new .. L-1, L = seq_lens[s]) the raw key and value are convolved with
+ * the 3 previous raw tokens (from the rolling state, then from the earlier
+ * new tokens), rounded to bf16 and written to their slot of the paged cache:
+ * block block_table[s, pos/128], slot pos%128.  The state then holds the last
+ * 3 raw tokens.  Arithmetic: fp32, taps applied oldest first
+ * (w3*x[t-3] + w2*x[t-2] + w1*x[t-1] + w0*x[t], fused multiply-adds), one
+ * bf16 rounding.
+ * -------------------------------------------------------------------------- */
+typedef struct {
+    const void *k_new;           /* device [S, n_new, Hkv, d] bf16 raw keys */
+    const void *v_new;           /* device [S, n_new, Hkv, d] bf16 raw values */
+    const float *w_k;            /* device [Hkv*d, 4] fp32 key taps (tap 0 = current) */
+    const float *w_v;            /* device [Hkv*d, 4] fp32 value taps */
+    void *k_state;               /* device [S, 3, Hkv*d] bf16 raw key history, oldest first; updated */
+    void *v_state;               /* device [S, 3, Hkv*d] bf16 raw value history; updated */
+    void *k_cache;               /* device [num_blocks, Hkv, 128, d] bf16; new slots written */
+    void *v_cache;               /* device [num_blocks, Hkv, 128, d] bf16 */
+    const int32_t *block_table;  /* device [S, max_blocks] */
+    const int32_t *seq_lens;     /* device [S], lengths after the append, >= n_new */
+    int32_t *status;             /* device int32 or NULL */
+    int32_t num_seqs;            /* S >= 0 (0 = nothing to do) */
+    int32_t n_new;               /* new tokens per sequence, 1..64 */
+    int32_t num_kv_heads;        /* Hkv >= 1 */
+    int32_t head_dim;            /* d, must be 128 */
+    int32_t max_blocks;          /* columns of block_table */
+    int32_t num_blocks;          /* blocks in the cache pool */
+} inkling_sconv_params;
+
+inkling_status inkling_sconv_kv(const inkling_sconv_params *p, inkling_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * inkling_attn_prefill — prefill attention with the sconv fused into the
+ * key/value tile load (Overview, "Attention" and "Short convolution"; the
+ * relative term is the FA4 "sheared-bias" kernel named in section
+ * Performance).
+ *
+ * Every query row i of every sequence attends to keys j of the same sequence
+ * with 0 <= i-j (< window when window > 0).  Keys and values are the sconv of
+ * k_raw / v_raw with zero history before t = 0, rounded to bf16, exactly as
+ * inkling_sconv_kv would write them.  Logits use scale 1/sqrt(128) on q.k and
+ * add bias[h, min(i-j, d_max)] unscaled; softmax and accumulation are fp32,
+ * probabilities enter the P.V product as bf16, the output is rounded to bf16.
+ * -------------------------------------------------------------------------- */
+typedef struct {
+    const void *q;        /* device [B, T, Hq, d] bf16 */
+    const void *k_raw;    /* device [B, T, Hkv, d] bf16, before sconv */
+    const void *v_raw;    /* device [B, T, Hkv, d] bf16, before sconv */
+    const float *w_k;     /* device [Hkv*d, 4] fp32 */
+    const float *w_v;     /* device [Hkv*d, 4] fp32 */
+    const float *bias;    /* device [Hq, d_max+1] fp32 relative-position table */
+    void *out;            /* device [B, T, Hq, d] bf16 */
+    float *lse;           /* device [B, Hq, T] fp32 natural-log row logsumexp, or NULL */
+    int32_t *status;      /* device int32 or NULL */
+    int32_t batch;        /* B >= 0 */
+    int32_t seq_len;      /* T >= 0 */
+    int32_t num_q_heads;  /* Hq, a multiple of Hkv */
+    int32_t num_kv_heads; /* Hkv >= 1 */
+    int32_t head_dim;     /* d, must be 128 */
+    int32_t window;       /* 0 = full causal, else keys with i-j < window */
+    int32_t d_max;        /* bias table has d_max+1 entries per head, d_max >= 0 */
+} inkling_prefill_params;
+
+inkling_status inkling_attn_prefill(const inkling_prefill_params *p, inkling_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * inkling_attn_decode — single-token decode over the paged cache, split-KV.
+ *
+ * For sequence s with length L = seq_lens[s], the query q[s] sits at position
+ * L-1 and attends to positions max(0, L-window) .. L-1 (0 .. L-1 when
+ * window = 0), read through block_table, with the same logits as prefill.
+ * The key range of every sequence is cut into num_splits parts that run on
+ * separate thread blocks; their partial (max, sum, unnormalised output)
+ * triples go to the caller's workspace and a second kernel merges them.
+ * -------------------------------------------------------------------------- */
+typedef struct {
+    const void *q;               /* device [S, Hq, d] bf16 */
+    const void *k_cache;         /* device [num_blocks, Hkv, 128, d] bf16, post-sconv */
+    const void *v_cache;         /* device [num_blocks, Hkv, 128, d] bf16, post-sconv */
+    const int32_t *block_table;  /* device [S, max_blocks] */
+    const int32_t *seq_lens;     /* device [S], each in [1, max_blocks*128] */
+    const float *bias;           /* device [Hq, d_max+1] fp32 */
+    void *out;                   /* device [S, Hq, d] bf16 */
+    float *lse;                  /* device [S, Hq] fp32 or NULL */
+    int32_t *status;             /* device int32 or NULL */
+    int32_t num_seqs;            /* S >= 0 */
+    int32_t num_q_heads;         /* Hq = G * Hkv with 1 <= G <= 8 */
+    int32_t num_kv_heads;        /* Hkv >= 1 */
+    int32_t head_dim;            /* d, must be 128 */
+    int32_t max_blocks;          /* columns of block_table */
+    int32_t num_blocks;          /* blocks in the pool */
+    int32_t window;              /* 0 = full */
+    int32_t d_max;               /* >= 0 */
+    int32_t num_splits;          /* 0 = choose from the SM count, else 1..1024 */
+} inkling_decode_params;
+
+/* Workspace bytes inkling_attn_decode needs for num_splits splits (pass the
+ * value the call will use, or the result of inkling_attn_decode_num_splits).
+ * Returns 0 for invalid arguments. */
+size_t inkling_attn_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
+                                           int32_t num_splits);
+
+/* The split count inkling_attn_decode uses for these parameters (resolves
+ * num_splits = 0); returns 0 for invalid parameters. */
+int32_t inkling_attn_decode_num_splits(const inkling_decode_params *p);
+
+/* workspace: device, >= inkling_attn_decode_workspace_bytes(...) bytes, 16-byte
+ * aligned, contents need no initialisation; not used when the split count is 1. */
+inkling_status inkling_attn_decode(const inkling_decode_params *p, void *workspace,
+                                   size_t workspace_bytes, inkling_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* INKLING_H */

@@ -1,0 +1,19 @@
+"""Inkling decoder attention layer for NVIDIA B200 (sm_100a).
+
+The layer: a causal depthwise window-4 short convolution over keys and values,
+then grouped-query attention at head size 128 with a learned relative-position
+bias added to the logits, sliding-window or full causal.  The compute runs in
+libinkling.so (hand-written CUDA, C ABI in include/inkling.h); ``binding``
+marshals torch tensors into it and ``inputs`` draws seeded synthetic inputs.
+"""
+from .binding import (  # noqa: F401
+    attn_decode,
+    attn_prefill,
+    decode_num_splits,
+    decode_workspace_bytes,
+    load_library,
+    sconv_kv,
+)
+
+__all__ = ["attn_prefill", "attn_decode", "sconv_kv", "decode_num_splits",
+           "decode_workspace_bytes", "load_library"]

@@ -1,0 +1,249 @@
+"""Python binding of libinkling (ctypes): argument marshalling only.
+
+Every step of the layer runs in the library's CUDA kernels; this module checks
+torch tensors (device, dtype, shape, contiguity), turns them into pointers and
+sizes, and calls the C ABI declared in include/inkling.h on the current torch
+stream.  It never computes a result itself and has no CPU fallback: if the
+library is missing or the device is not sm_100, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libinkling.so")
+
+INKLING_OK, INKLING_ERR_INVALID, INKLING_ERR_UNSUPPORTED, INKLING_ERR_CUDA = 0, 1, 2, 3
+STATUS_TIMEOUT, STATUS_BAD_BLOCK, STATUS_BAD_LENGTH = 1, 2, 4
+HEAD_DIM = 128
+BLOCK_SIZE = 128
+
+EXPORTED = (
+    "inkling_last_error",
+    "inkling_version",
+    "inkling_sconv_kv",
+    "inkling_attn_prefill",
+    "inkling_attn_decode_workspace_bytes",
+    "inkling_attn_decode_num_splits",
+    "inkling_attn_decode",
+)
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int32
+
+
+class SconvParams(ctypes.Structure):
+    _fields_ = [("k_new", _P), ("v_new", _P), ("w_k", _P), ("w_v", _P), ("k_state", _P),
+                ("v_state", _P), ("k_cache", _P), ("v_cache", _P), ("block_table", _P),
+                ("seq_lens", _P), ("status", _P), ("num_seqs", _I), ("n_new", _I),
+                ("num_kv_heads", _I), ("head_dim", _I), ("max_blocks", _I), ("num_blocks", _I)]
+
+
+class PrefillParams(ctypes.Structure):
+    _fields_ = [("q", _P), ("k_raw", _P), ("v_raw", _P), ("w_k", _P), ("w_v", _P), ("bias", _P),
+                ("out", _P), ("lse", _P), ("status", _P), ("batch", _I), ("seq_len", _I),
+                ("num_q_heads", _I), ("num_kv_heads", _I), ("head_dim", _I), ("window", _I),
+                ("d_max", _I)]
+
+
+class DecodeParams(ctypes.Structure):
+    _fields_ = [("q", _P), ("k_cache", _P), ("v_cache", _P), ("block_table", _P),
+                ("seq_lens", _P), ("bias", _P), ("out", _P), ("lse", _P), ("status", _P),
+                ("num_seqs", _I), ("num_q_heads", _I), ("num_kv_heads", _I), ("head_dim", _I),
+                ("max_blocks", _I), ("num_blocks", _I), ("window", _I), ("d_max", _I),
+                ("num_splits", _I)]
+
+
+class InklingError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"libinkling error {code}: {msg}")
+        self.code = code
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libinkling.so and declare its signatures (raises if it is absent)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is not built: run `python -m relative_bias_sliding_b200.build`")
+        lib = ctypes.CDLL(path)
+        lib.inkling_last_error.restype = ctypes.c_char_p
+        lib.inkling_version.restype = ctypes.c_int
+        lib.inkling_sconv_kv.argtypes = [ctypes.POINTER(SconvParams), _P]
+        lib.inkling_sconv_kv.restype = ctypes.c_int
+        lib.inkling_attn_prefill.argtypes = [ctypes.POINTER(PrefillParams), _P]
+        lib.inkling_attn_prefill.restype = ctypes.c_int
+        lib.inkling_attn_decode_workspace_bytes.argtypes = [_I, _I, _I]
+        lib.inkling_attn_decode_workspace_bytes.restype = ctypes.c_size_t
+        lib.inkling_attn_decode_num_splits.argtypes = [ctypes.POINTER(DecodeParams)]
+        lib.inkling_attn_decode_num_splits.restype = _I
+        lib.inkling_attn_decode.argtypes = [ctypes.POINTER(DecodeParams), _P, ctypes.c_size_t, _P]
+        lib.inkling_attn_decode.restype = ctypes.c_int
+        _lib = lib
+        return lib
+
+
+def _check(code):
+    if code != INKLING_OK:
+        raise InklingError(code, load_library().inkling_last_error().decode())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev(t, dtype, name, ndim=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+    return t
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def sconv_kv(k_new, v_new, w_k, w_v, k_state, v_state, k_cache, v_cache, block_table, seq_lens,
+             status=None, stream=None):
+    """Decode-side sconv append (in place on the states and caches)."""
+    bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    _dev(k_new, bf, "k_new", 4), _dev(v_new, bf, "v_new", 4)
+    S, n_new, Hkv, d = k_new.shape
+    if v_new.shape != k_new.shape:
+        raise ValueError("k_new and v_new shapes differ")
+    for n, t in (("w_k", w_k), ("w_v", w_v)):
+        _dev(t, f32, n)
+        if t.shape != (Hkv * d, 4):
+            raise ValueError(f"{n} must be [{Hkv * d}, 4]")
+    for n, t in (("k_state", k_state), ("v_state", v_state)):
+        _dev(t, bf, n)
+        if t.shape != (S, 3, Hkv * d):
+            raise ValueError(f"{n} must be [{S}, 3, {Hkv * d}]")
+    for n, t in (("k_cache", k_cache), ("v_cache", v_cache)):
+        _dev(t, bf, n, 4)
+        if t.shape[1:] != (Hkv, BLOCK_SIZE, d):
+            raise ValueError(f"{n} must be [num_blocks, {Hkv}, 128, {d}]")
+    _dev(block_table, i32, "block_table", 2), _dev(seq_lens, i32, "seq_lens", 1)
+    _dev(status, i32, "status")
+    p = SconvParams(_ptr(k_new), _ptr(v_new), _ptr(w_k), _ptr(w_v), _ptr(k_state), _ptr(v_state),
+                    _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens), _ptr(status),
+                    S, n_new, Hkv, d, block_table.shape[1], k_cache.shape[0])
+    _check(load_library().inkling_sconv_kv(ctypes.byref(p), _stream(stream)))
+
+
+def attn_prefill(q, k_raw, v_raw, w_k, w_v, bias, window=0, out=None, lse=None, status=None,
+                 stream=None):
+    """Prefill attention with fused sconv; returns ``out`` [B, T, Hq, d] bf16."""
+    bf, f32 = torch.bfloat16, torch.float32
+    _dev(q, bf, "q", 4), _dev(k_raw, bf, "k_raw", 4), _dev(v_raw, bf, "v_raw", 4)
+    B, T, Hq, d = q.shape
+    Hkv = k_raw.shape[2]
+    if k_raw.shape != (B, T, Hkv, d) or v_raw.shape != k_raw.shape:
+        raise ValueError("k_raw / v_raw must be [B, T, Hkv, d] matching q")
+    for n, t in (("w_k", w_k), ("w_v", w_v)):
+        _dev(t, f32, n)
+        if t.shape != (Hkv * d, 4):
+            raise ValueError(f"{n} must be [{Hkv * d}, 4]")
+    _dev(bias, f32, "bias", 2)
+    if bias.shape[0] != Hq:
+        raise ValueError("bias must be [Hq, d_max+1]")
+    d_max = bias.shape[1] - 1
+    if out is None:
+        out = torch.empty_like(q)
+    _dev(out, bf, "out", 4)
+    if out.shape != q.shape:
+        raise ValueError("out must match q")
+    if lse is not None:
+        _dev(lse, f32, "lse", 3)
+        if lse.shape != (B, Hq, T):
+            raise ValueError("lse must be [B, Hq, T]")
+    _dev(status, torch.int32, "status")
+    p = PrefillParams(_ptr(q), _ptr(k_raw), _ptr(v_raw), _ptr(w_k), _ptr(w_v), _ptr(bias),
+                      _ptr(out), _ptr(lse), _ptr(status), B, T, Hq, Hkv, d, int(window), d_max)
+    _check(load_library().inkling_attn_prefill(ctypes.byref(p), _stream(stream)))
+    return out
+
+
+def _decode_params(q, k_cache, v_cache, block_table, seq_lens, bias, window, out, lse, status,
+                   num_splits):
+    bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    _dev(q, bf, "q", 3)
+    S, Hq, d = q.shape
+    _dev(k_cache, bf, "k_cache", 4), _dev(v_cache, bf, "v_cache", 4)
+    if k_cache.shape != v_cache.shape or k_cache.shape[2] != BLOCK_SIZE or k_cache.shape[3] != d:
+        raise ValueError("caches must be [num_blocks, Hkv, 128, d] and equal")
+    Hkv = k_cache.shape[1]
+    _dev(block_table, i32, "block_table", 2), _dev(seq_lens, i32, "seq_lens", 1)
+    if block_table.shape[0] != S or seq_lens.shape[0] != S:
+        raise ValueError("block_table / seq_lens must have num_seqs rows")
+    _dev(bias, f32, "bias", 2)
+    if bias.shape[0] != Hq:
+        raise ValueError("bias must be [Hq, d_max+1]")
+    _dev(out, bf, "out", 3)
+    if out.shape != q.shape:
+        raise ValueError("out must match q")
+    if lse is not None:
+        _dev(lse, f32, "lse", 2)
+        if lse.shape != (S, Hq):
+            raise ValueError("lse must be [S, Hq]")
+    _dev(status, i32, "status")
+    return DecodeParams(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
+                        _ptr(bias), _ptr(out), _ptr(lse), _ptr(status), S, Hq, Hkv, d,
+                        block_table.shape[1], k_cache.shape[0], int(window), bias.shape[1] - 1,
+                        int(num_splits))
+
+
+def decode_num_splits(q, k_cache, v_cache, block_table, seq_lens, bias, window=0, num_splits=0):
+    """Split count the decode call will use (resolves num_splits=0)."""
+    out = torch.empty_like(q)
+    p = _decode_params(q, k_cache, v_cache, block_table, seq_lens, bias, window, out, None, None,
+                       num_splits)
+    n = load_library().inkling_attn_decode_num_splits(ctypes.byref(p))
+    if n <= 0:
+        raise InklingError(INKLING_ERR_INVALID, load_library().inkling_last_error().decode())
+    return int(n)
+
+
+def decode_workspace_bytes(num_seqs, num_q_heads, num_splits):
+    return int(load_library().inkling_attn_decode_workspace_bytes(num_seqs, num_q_heads,
+                                                                   num_splits))
+
+
+def attn_decode(q, k_cache, v_cache, block_table, seq_lens, bias, window=0, out=None, lse=None,
+                workspace=None, num_splits=0, status=None, stream=None):
+    """Single-token paged decode; returns ``out`` [S, Hq, d] bf16.  ``workspace``
+    (uint8 CUDA tensor) is allocated here by torch when not given."""
+    if out is None:
+        out = torch.empty_like(q)
+    p = _decode_params(q, k_cache, v_cache, block_table, seq_lens, bias, window, out, lse, status,
+                       num_splits)
+    lib = load_library()
+    splits = lib.inkling_attn_decode_num_splits(ctypes.byref(p))
+    if splits <= 0:
+        _check(INKLING_ERR_INVALID if not lib.inkling_last_error() else INKLING_ERR_INVALID)
+    need = lib.inkling_attn_decode_workspace_bytes(p.num_seqs, p.num_q_heads, splits)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _dev(workspace, torch.uint8, "workspace")
+    _check(lib.inkling_attn_decode(ctypes.byref(p), _ptr(workspace), workspace.numel(),
+                                   _stream(stream)))
+    return out

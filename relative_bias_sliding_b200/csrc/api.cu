@@ -1,0 +1,263 @@
+// api.cu — the extern "C" boundary of libinkling: argument validation, TMA
+// descriptor encoding, launches on the caller's stream.  No allocation, no
+// synchronisation, no state besides the per-thread error message.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace inkling {
+cudaError_t launch_sconv_kv(const inkling_sconv_params &p, cudaStream_t stream);
+cudaError_t launch_attn_prefill(const inkling_prefill_params &p, const CUtensorMap *maps,
+                                cudaStream_t stream);
+cudaError_t launch_attn_decode(const inkling_decode_params &p, int splits, void *workspace,
+                               const CUtensorMap &tm_k, const CUtensorMap &tm_v,
+                               cudaStream_t stream);
+}  // namespace inkling
+
+using namespace inkling;
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+inkling_status fail(inkling_status st, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+inkling_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(INKLING_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (EncodeTiledFn)p;
+    });
+    return fn;
+}
+
+// bf16 tensor map, 128-byte swizzle, rank <= 4; dims/strides in elements/bytes
+inkling_status make_map(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims,
+                        const cuuint64_t *strides_bytes, const cuuint32_t *box) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(INKLING_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(base),
+                    dims, strides_bytes, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(INKLING_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return INKLING_OK;
+}
+
+// sm_100 check for the current device (cached per device)
+inkling_status check_device(int *num_sms) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    static int major[64], sms[64];
+    if (dev < 0 || dev >= 64) return fail(INKLING_ERR_UNSUPPORTED, "device index %d", dev);
+    if (major[dev] == 0) {
+        int mj = 0, n = 0;
+        e = cudaDeviceGetAttribute(&mj, cudaDevAttrComputeCapabilityMajor, dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+        e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+        sms[dev] = n;
+        major[dev] = mj;
+    }
+    if (major[dev] != 10)
+        return fail(INKLING_ERR_UNSUPPORTED, "libinkling is built for sm_100a (B200); device %d has "
+                                             "compute capability %d.x", dev, major[dev]);
+    if (num_sms) *num_sms = sms[dev];
+    return INKLING_OK;
+}
+
+int decode_splits(const inkling_decode_params &p, int num_sms) {
+    if (p.num_splits > 0) return p.num_splits;
+    const long max_keys = (long)p.max_blocks * 128;
+    const long keys = p.window > 0 ? (p.window < max_keys ? p.window : max_keys) : max_keys;
+    const long chunks = (keys + 63) / 64 + 1;
+    const long units = (long)p.num_seqs * p.num_kv_heads;
+    long s = (8L * num_sms + units - 1) / units;  // about 4 waves of 2 blocks per SM
+    long cap = chunks / 8;                        // at least ~8 chunks (512 keys) per split
+    if (cap < 1) cap = 1;
+    if (s > cap) s = cap;
+    if (s > 1024) s = 1024;
+    if (s < 1) s = 1;
+    return (int)s;
+}
+
+inkling_status validate_decode(const inkling_decode_params *p) {
+    if (!p) return fail(INKLING_ERR_INVALID, "params is NULL");
+    if (p->num_seqs < 0 || p->num_q_heads < 1 || p->num_kv_heads < 1)
+        return fail(INKLING_ERR_INVALID, "num_seqs must be >= 0 and head counts >= 1");
+    if (p->head_dim != INKLING_HEAD_DIM)
+        return fail(INKLING_ERR_UNSUPPORTED, "head_dim %d (only 128 is implemented)", p->head_dim);
+    if (p->num_q_heads % p->num_kv_heads)
+        return fail(INKLING_ERR_INVALID, "num_q_heads %% num_kv_heads != 0");
+    if (p->num_q_heads / p->num_kv_heads > 8)
+        return fail(INKLING_ERR_UNSUPPORTED, "decode supports at most 8 query heads per kv head");
+    if (p->max_blocks < 1 || p->num_blocks < 1)
+        return fail(INKLING_ERR_INVALID, "max_blocks and num_blocks must be >= 1");
+    if ((long)p->max_blocks * 128 > (1L << 30))
+        return fail(INKLING_ERR_UNSUPPORTED, "max_blocks * 128 exceeds 2^30 tokens");
+    if ((long)p->num_blocks * p->num_kv_heads * 128 >= (1L << 31))
+        return fail(INKLING_ERR_UNSUPPORTED, "cache pool rows exceed 2^31");
+    if (p->window < 0 || p->d_max < 0) return fail(INKLING_ERR_INVALID, "window and d_max must be >= 0");
+    if (p->num_splits < 0 || p->num_splits > 1024)
+        return fail(INKLING_ERR_INVALID, "num_splits must be in [0, 1024]");
+    if (p->num_seqs == 0) return INKLING_OK;
+    if (!p->q || !p->k_cache || !p->v_cache || !p->block_table || !p->seq_lens || !p->bias || !p->out)
+        return fail(INKLING_ERR_INVALID, "a required pointer is NULL");
+    if (!aligned16(p->q) || !aligned16(p->k_cache) || !aligned16(p->v_cache) || !aligned16(p->out))
+        return fail(INKLING_ERR_INVALID, "q, caches and out must be 16-byte aligned");
+    if (((uintptr_t)p->bias & 3u) != 0) return fail(INKLING_ERR_INVALID, "bias must be 4-byte aligned");
+    return INKLING_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *inkling_last_error(void) { return g_err; }
+
+int inkling_version(void) { return 100; }
+
+inkling_status inkling_sconv_kv(const inkling_sconv_params *p, inkling_stream_t stream) {
+    g_err[0] = 0;
+    if (!p) return fail(INKLING_ERR_INVALID, "params is NULL");
+    if (p->num_seqs < 0 || p->num_kv_heads < 1)
+        return fail(INKLING_ERR_INVALID, "num_seqs must be >= 0, num_kv_heads >= 1");
+    if (p->head_dim != INKLING_HEAD_DIM)
+        return fail(INKLING_ERR_UNSUPPORTED, "head_dim %d (only 128 is implemented)", p->head_dim);
+    if (p->n_new < 1 || p->n_new > 64) return fail(INKLING_ERR_INVALID, "n_new must be in [1, 64]");
+    if (p->max_blocks < 1 || p->num_blocks < 1)
+        return fail(INKLING_ERR_INVALID, "max_blocks and num_blocks must be >= 1");
+    if ((long)p->max_blocks * 128 > (1L << 30))
+        return fail(INKLING_ERR_UNSUPPORTED, "max_blocks * 128 exceeds 2^30 tokens");
+    if (p->num_seqs == 0) return INKLING_OK;
+    if (!p->k_new || !p->v_new || !p->w_k || !p->w_v || !p->k_state || !p->v_state || !p->k_cache ||
+        !p->v_cache || !p->block_table || !p->seq_lens)
+        return fail(INKLING_ERR_INVALID, "a required pointer is NULL");
+    if (!aligned16(p->k_new) || !aligned16(p->v_new) || !aligned16(p->w_k) || !aligned16(p->w_v) ||
+        !aligned16(p->k_state) || !aligned16(p->v_state) || !aligned16(p->k_cache) ||
+        !aligned16(p->v_cache))
+        return fail(INKLING_ERR_INVALID, "tensors must be 16-byte aligned");
+    inkling_status st = check_device(nullptr);
+    if (st != INKLING_OK) return st;
+    cudaError_t e = launch_sconv_kv(*p, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "sconv_kv launch");
+    return INKLING_OK;
+}
+
+inkling_status inkling_attn_prefill(const inkling_prefill_params *p, inkling_stream_t stream) {
+    g_err[0] = 0;
+    if (!p) return fail(INKLING_ERR_INVALID, "params is NULL");
+    if (p->batch < 0 || p->seq_len < 0 || p->num_q_heads < 1 || p->num_kv_heads < 1)
+        return fail(INKLING_ERR_INVALID, "batch, seq_len must be >= 0 and head counts >= 1");
+    if (p->head_dim != INKLING_HEAD_DIM)
+        return fail(INKLING_ERR_UNSUPPORTED, "head_dim %d (only 128 is implemented)", p->head_dim);
+    if (p->num_q_heads % p->num_kv_heads)
+        return fail(INKLING_ERR_INVALID, "num_q_heads %% num_kv_heads != 0");
+    if (p->window < 0 || p->d_max < 0) return fail(INKLING_ERR_INVALID, "window and d_max must be >= 0");
+    if (p->seq_len > (1 << 30)) return fail(INKLING_ERR_UNSUPPORTED, "seq_len above 2^30");
+    const long blocks = (long)p->batch * p->num_q_heads * ((p->seq_len + 255) / 256);
+    if (blocks > 0x7fffffffL) return fail(INKLING_ERR_UNSUPPORTED, "grid too large");
+    if (blocks == 0) return INKLING_OK;
+    if (!p->q || !p->k_raw || !p->v_raw || !p->w_k || !p->w_v || !p->bias || !p->out)
+        return fail(INKLING_ERR_INVALID, "a required pointer is NULL");
+    if (!aligned16(p->q) || !aligned16(p->k_raw) || !aligned16(p->v_raw) || !aligned16(p->w_k) ||
+        !aligned16(p->w_v) || !aligned16(p->out))
+        return fail(INKLING_ERR_INVALID, "q, k_raw, v_raw, taps and out must be 16-byte aligned");
+    inkling_status st = check_device(nullptr);
+    if (st != INKLING_OK) return st;
+
+    const cuuint64_t T = (cuuint64_t)p->seq_len, B = (cuuint64_t)p->batch;
+    const cuuint64_t Hq = (cuuint64_t)p->num_q_heads, Hkv = (cuuint64_t)p->num_kv_heads;
+    CUtensorMap maps[5];
+    {
+        // q [B, T, Hq, 128] seen as (d, T, Hq, B)
+        cuuint64_t dims[4] = {128, T, Hq, B};
+        cuuint64_t str[3] = {Hq * 256, 256, T * Hq * 256};
+        cuuint32_t box[4] = {64, 128, 1, 1};
+        if ((st = make_map(&maps[0], p->q, 4, dims, str, box)) != INKLING_OK) return st;
+    }
+    const void *kv[2] = {p->k_raw, p->v_raw};
+    for (int w = 0; w < 2; ++w) {
+        // raw keys / values [B, T, Hkv, 128] seen as (d, T, Hkv, B): a 128-row
+        // tile box and an 8-row history box
+        cuuint64_t dims[4] = {128, T, Hkv, B};
+        cuuint64_t str[3] = {Hkv * 256, 256, T * Hkv * 256};
+        cuuint32_t box_t[4] = {64, 128, 1, 1};
+        cuuint32_t box_h[4] = {64, 8, 1, 1};
+        if ((st = make_map(&maps[1 + 2 * w], kv[w], 4, dims, str, box_t)) != INKLING_OK) return st;
+        if ((st = make_map(&maps[2 + 2 * w], kv[w], 4, dims, str, box_h)) != INKLING_OK) return st;
+    }
+    cudaError_t e = launch_attn_prefill(*p, maps, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "attn_prefill launch");
+    return INKLING_OK;
+}
+
+size_t inkling_attn_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_splits) {
+    if (num_seqs < 0 || num_q_heads < 1 || num_splits < 1 || num_splits > 1024) return 0;
+    if (num_splits == 1) return 16;  // no partials; any non-NULL pointer will do
+    return (size_t)num_seqs * num_q_heads * num_splits * (128 + 2) * sizeof(float);
+}
+
+int32_t inkling_attn_decode_num_splits(const inkling_decode_params *p) {
+    if (validate_decode(p) != INKLING_OK) return 0;
+    int sms = 0;
+    if (check_device(&sms) != INKLING_OK) return 0;
+    return decode_splits(*p, sms);
+}
+
+inkling_status inkling_attn_decode(const inkling_decode_params *p, void *workspace,
+                                   size_t workspace_bytes, inkling_stream_t stream) {
+    g_err[0] = 0;
+    inkling_status st = validate_decode(p);
+    if (st != INKLING_OK) return st;
+    if (p->num_seqs == 0) return INKLING_OK;
+    int sms = 0;
+    if ((st = check_device(&sms)) != INKLING_OK) return st;
+    const int splits = decode_splits(*p, sms);
+    if (splits > 1) {
+        const size_t need = inkling_attn_decode_workspace_bytes(p->num_seqs, p->num_q_heads, splits);
+        if (!workspace || workspace_bytes < need)
+            return fail(INKLING_ERR_INVALID, "workspace of %zu bytes given, %zu needed for %d splits",
+                        workspace_bytes, need, splits);
+        if (!aligned16(workspace)) return fail(INKLING_ERR_INVALID, "workspace must be 16-byte aligned");
+    }
+    CUtensorMap tm_k, tm_v;
+    const cuuint64_t rows = (cuuint64_t)p->num_blocks * p->num_kv_heads * 128;
+    cuuint64_t dims[2] = {128, rows};
+    cuuint64_t str[1] = {256};
+    cuuint32_t box[2] = {64, 64};
+    if ((st = make_map(&tm_k, p->k_cache, 2, dims, str, box)) != INKLING_OK) return st;
+    if ((st = make_map(&tm_v, p->v_cache, 2, dims, str, box)) != INKLING_OK) return st;
+    cudaError_t e = launch_attn_decode(*p, splits, workspace, tm_k, tm_v, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "attn_decode launch");
+    return INKLING_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,384 @@
+// attn_decode.cu — single-token decode over the paged KV cache, split-KV
+// (vLLM Recipes "thinkingmachines/Inkling": Overview "Attention" bullet —
+// GQA at head size 128 with a learned relative-position term added to the
+// pre-softmax logits, sliding-window or full layers; 128-token cache blocks
+// from the `--block-size 128` launch option; 1M-token context).
+//
+// Design (HBM-bound: each key/value byte is read once, 8 query heads share it):
+//  * grid = num_seqs x Hkv x num_splits thread blocks; a block owns one kv head
+//    of one sequence and a contiguous run of 64-key chunks of its key range.
+//  * warp 4 is the producer: it reads block ids from the block table (one
+//    coalesced load per 32 blocks) and issues TMA loads of 64-key halves of a
+//    cache block (keys and values, 128-byte swizzled, 32 KB per stage) into a
+//    3-stage mbarrier ring.
+//  * warps 0-3 each take 16 keys of a chunk: S = Q K^T with mma.sync m16n8k16
+//    (rows = the 8 query heads of the group, padded to 16), logits in log2
+//    units plus bias, online softmax with quad shuffles, O += P V with the
+//    P accumulator fragment reused as the A operand and V read by
+//    ldmatrix.trans.  No tcgen05 here: at 8 flop/byte the tensor work is a
+//    small fraction of the stream time and mma.sync keeps it in registers.
+//  * the 4 warps merge through shared memory; with one split the block writes
+//    the bf16 output, otherwise an unnormalised partial (m, l, O) that
+//    decode_combine_kernel merges.
+#include "common.cuh"
+
+namespace inkling {
+
+constexpr int kDecStages = 3;
+constexpr int kDecStageBytes = 32768;  // 64 keys x 128 d x bf16, keys + values
+constexpr int kDecSmem = kDecStages * kDecStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+
+struct DecodeArgs {
+    const uint16_t *q;
+    const int32_t *block_table;
+    const int32_t *seq_lens;
+    const float *bias;
+    uint16_t *out;
+    float *lse;
+    float *part_o;   // [S, Hq, splits, 128]
+    float *part_ml;  // [S, Hq, splits, 2] (max in log2 units, sum)
+    int32_t *status;
+    int S, Hq, Hkv, G, max_blocks, num_blocks, window, d_max, splits;
+};
+
+INK_DEV void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+INK_DEV void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+INK_DEV void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// byte offset of (row r, 16-byte chunk cc of a 128-byte row) in a
+// 128-byte-swizzled tile whose base is 1024-byte aligned
+INK_DEV uint32_t sw128_off(int r, int cc) { return (uint32_t)(r * 128 + ((cc ^ (r & 7)) << 4)); }
+
+__global__ void __launch_bounds__(160, 2)
+decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const DecodeArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint64_t *full = (uint64_t *)(smem + kDecStages * kDecStageBytes);
+    uint64_t *empty = full + kDecStages;
+    volatile int *abort_flag = (volatile int *)(empty + kDecStages);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int s = blockIdx.x % a.S;
+    const int kvh = (blockIdx.x / a.S) % a.Hkv;
+    const int split = blockIdx.x / (a.S * a.Hkv);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kDecStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 4);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    // key range of this sequence and this split, in 64-key chunks
+    const int L = a.seq_lens[s];
+    const bool bad_len = (L < 1 || L > a.max_blocks * 128);
+    const int lo = (a.window > 0) ? max(0, L - a.window) : 0;
+    int ca = 0, cb = 0;
+    if (!bad_len) {
+        const int c_lo = lo >> 6, c_hi = (L + 63) >> 6;
+        const int per = (c_hi - c_lo + a.splits - 1) / a.splits;
+        ca = min(c_hi, c_lo + split * per);
+        cb = min(c_hi, ca + per);
+    } else if (threadIdx.x == 0 && split == 0 && kvh == 0) {
+        report_status(a.status, INKLING_STATUS_BAD_LENGTH);
+    }
+
+    if (warp == 4) {
+        // ------------------------------------------------------- producer --
+        int cur_batch = -1, my_id = 0, issued = 0;
+        for (int c = ca; c < cb; ++c) {
+            const int bi = c >> 1;
+            if ((bi >> 5) != cur_batch) {
+                cur_batch = bi >> 5;
+                const int idx = cur_batch * 32 + lane;
+                my_id = (idx < a.max_blocks) ? a.block_table[(long)s * a.max_blocks + idx] : 0;
+            }
+            int blk = __shfl_sync(0xffffffffu, my_id, bi & 31);
+            int ok = 1;
+            if (lane == 0) {
+                const int k = c - ca, st = k % kDecStages;
+                ok = mbar_wait(&empty[st], ((k / kDecStages) & 1) ^ 1, abort_flag, a.status);
+                if (ok) {
+                    if (blk < 0 || blk >= a.num_blocks) {
+                        report_status(a.status, INKLING_STATUS_BAD_BLOCK);
+                        blk = 0;  // keep the pipeline running on a valid block
+                    }
+                    const int row = (blk * a.Hkv + kvh) * 128 + (c & 1) * 64;
+                    uint8_t *kb = smem + st * kDecStageBytes;
+                    mbar_arrive_expect_tx(&full[st], kDecStageBytes);
+                    tma_load_2d(kb, &tm_k, &full[st], 0, row);
+                    tma_load_2d(kb + 8192, &tm_k, &full[st], 64, row);
+                    tma_load_2d(kb + 16384, &tm_v, &full[st], 0, row);
+                    tma_load_2d(kb + 24576, &tm_v, &full[st], 64, row);
+                    ++issued;
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+        }
+        // drain: every load issued has landed before the block may exit
+        if (lane == 0) {
+            for (int k = max(0, issued - kDecStages); k < issued; ++k)
+                mbar_wait(&full[k % kDecStages], (k / kDecStages) & 1, nullptr, a.status);
+        }
+    } else {
+        // --------------------------------------------------------- compute --
+        const int g = lane >> 2, t = lane & 3;
+        const bool row_ok = g < a.G;
+        const int h = kvh * a.G + (row_ok ? g : 0);
+        const uint16_t *qrow = a.q + ((long)s * a.Hq + h) * 128;
+        uint32_t qa[8][4];
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            qa[ks][0] = row_ok ? *(const uint32_t *)(qrow + 16 * ks + 2 * t) : 0u;
+            qa[ks][2] = row_ok ? *(const uint32_t *)(qrow + 16 * ks + 8 + 2 * t) : 0u;
+            qa[ks][1] = 0u;
+            qa[ks][3] = 0u;
+        }
+        const float kLog2e = 1.4426950408889634f;
+        const float c1 = kLog2e * 0.08838834764831845f;  // log2(e) / sqrt(128)
+        const float *bias_h = a.bias + (long)h * (a.d_max + 1);
+
+        float o[16][4];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+        float m = -INFINITY, l = 0.f;
+
+        const uint32_t sbase = smem_u32(smem);
+        for (int c = ca; c < cb; ++c) {
+            const int k = c - ca, st = k % kDecStages;
+            // bias for this thread's 4 keys, fetched before the wait
+            float bv[2][2];
+            int jj[2][2];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int j = c * 64 + warp * 16 + nt * 8 + 2 * t + e;
+                    jj[nt][e] = j;
+                    const int dist = L - 1 - j;
+                    const bool ok = row_ok && j >= lo && j < L;
+                    bv[nt][e] = ok ? __ldg(bias_h + min(dist, a.d_max)) : 0.f;
+                }
+            if (!mbar_wait_warp(&full[st], (k / kDecStages) & 1, abort_flag, a.status)) break;
+
+            const uint32_t kst = sbase + st * kDecStageBytes;
+            const uint32_t vst = kst + 16384;
+            // S = Q K^T over this warp's 16 keys (two n-tiles of 8)
+            float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            {
+                const int r = warp * 16 + ((lane >> 4) & 1) * 8 + (lane & 7);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const int cc = 2 * (ks & 3) + ((lane >> 3) & 1);
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4(kst + (ks >> 2) * 8192 + sw128_off(r, cc), b0, b1, b2, b3);
+                    mma16816(sacc[0], qa[ks], b0, b1);
+                    mma16816(sacc[1], qa[ks], b2, b3);
+                }
+            }
+            // logits (log2 units), mask, online softmax
+            float x[2][2];
+            float mx = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int j = jj[nt][e];
+                    const bool ok = row_ok && j >= lo && j < L;
+                    x[nt][e] = ok ? fmaf(sacc[nt][e], c1, bv[nt][e] * kLog2e) : -INFINITY;
+                    mx = fmaxf(mx, x[nt][e]);
+                }
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            const float m_new = fmaxf(m, mx);
+            const float alpha = (m == -INFINITY) ? 0.f : ex2(m - m_new);
+            float p[2][2], psum = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    p[nt][e] = (x[nt][e] == -INFINITY) ? 0.f : ex2(x[nt][e] - m_new);
+                    psum += p[nt][e];
+                }
+            l = l * alpha + psum;
+            m = m_new;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                o[i][0] *= alpha;
+                o[i][1] *= alpha;
+            }
+            uint32_t pa[4];
+            pa[0] = pack_bf16(p[0][0], p[0][1]);
+            pa[1] = 0u;
+            pa[2] = pack_bf16(p[1][0], p[1][1]);
+            pa[3] = 0u;
+            // O += P V over the 16 keys, 16 n-tiles of 8 head-dim columns
+            {
+                const int r = warp * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
+#pragma unroll
+                for (int mm = 0; mm < 8; ++mm) {
+                    const int ch = 2 * mm + (lane >> 4);  // 16-byte chunk of d
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4_t(vst + (ch >> 3) * 8192 + sw128_off(r, ch & 7), b0, b1, b2, b3);
+                    mma16816(o[2 * mm], pa, b0, b1);
+                    mma16816(o[2 * mm + 1], pa, b2, b3);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
+        }
+        l += __shfl_xor_sync(0xffffffffu, l, 1);
+        l += __shfl_xor_sync(0xffffffffu, l, 2);
+
+        // merge the 4 warps through shared memory (the ring is idle now)
+        named_bar_sync(1, 128);
+        float *red_o = (float *)smem;                  // [4][8][128]
+        float *red_ml = red_o + 4 * 8 * 128;           // [4][8][2]
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            red_o[(warp * 8 + g) * 128 + i * 8 + 2 * t] = o[i][0];
+            red_o[(warp * 8 + g) * 128 + i * 8 + 2 * t + 1] = o[i][1];
+        }
+        if (t == 0) {
+            red_ml[(warp * 8 + g) * 2] = m;
+            red_ml[(warp * 8 + g) * 2 + 1] = l;
+        }
+        named_bar_sync(1, 128);
+        const int u = threadIdx.x;  // 0..127
+        const int gg = u >> 4, d0 = (u & 15) * 8;
+        if (gg < a.G && !*abort_flag) {
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) M = fmaxf(M, red_ml[(w * 8 + gg) * 2]);
+            float f[4], Ls = 0.f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const float mw = red_ml[(w * 8 + gg) * 2];
+                f[w] = (mw == -INFINITY) ? 0.f : ex2(mw - M);
+                Ls += f[w] * red_ml[(w * 8 + gg) * 2 + 1];
+            }
+            float acc[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                float v = 0.f;
+#pragma unroll
+                for (int w = 0; w < 4; ++w) v = fmaf(f[w], red_o[(w * 8 + gg) * 128 + d0 + e], v);
+                acc[e] = v;
+            }
+            const int hh = kvh * a.G + gg;
+            if (a.splits == 1) {
+                const float inv = (Ls > 0.f) ? 1.f / Ls : 0.f;
+                uint4 pk;
+                pk.x = pack_bf16(acc[0] * inv, acc[1] * inv);
+                pk.y = pack_bf16(acc[2] * inv, acc[3] * inv);
+                pk.z = pack_bf16(acc[4] * inv, acc[5] * inv);
+                pk.w = pack_bf16(acc[6] * inv, acc[7] * inv);
+                *(uint4 *)(a.out + ((long)s * a.Hq + hh) * 128 + d0) = pk;
+                if (a.lse && (u & 15) == 0)
+                    a.lse[(long)s * a.Hq + hh] =
+                        (Ls > 0.f) ? (M + __log2f(Ls)) * 0.6931471805599453f : -INFINITY;
+            } else {
+                const long pi = ((long)s * a.Hq + hh) * a.splits + split;
+                float4 *po = (float4 *)(a.part_o + pi * 128 + d0);
+                po[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                po[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+                if ((u & 15) == 0) {
+                    a.part_ml[pi * 2] = M;
+                    a.part_ml[pi * 2 + 1] = Ls;
+                }
+            }
+        }
+    }
+    __syncthreads();
+}
+
+// One warp per (sequence, query head): log-sum-exp merge of the splits.
+__global__ void __launch_bounds__(128)
+decode_combine_kernel(const float *__restrict__ part_o, const float *__restrict__ part_ml,
+                      uint16_t *__restrict__ out, float *__restrict__ lse, int pairs, int splits) {
+    const int pair = blockIdx.x * 4 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (pair >= pairs) return;
+    const float *ml = part_ml + (long)pair * splits * 2;
+    float M = -INFINITY;
+    for (int sp = lane; sp < splits; sp += 32) M = fmaxf(M, ml[sp * 2]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float Ls = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 *po = (const float4 *)(part_o + (long)pair * splits * 128) + lane;
+    for (int sp = 0; sp < splits; ++sp) {
+        const float msp = ml[sp * 2];
+        if (msp == -INFINITY) continue;
+        const float f = ex2(msp - M);
+        Ls = fmaf(f, ml[sp * 2 + 1], Ls);
+        const float4 v = po[sp * 32];
+        acc.x = fmaf(f, v.x, acc.x);
+        acc.y = fmaf(f, v.y, acc.y);
+        acc.z = fmaf(f, v.z, acc.z);
+        acc.w = fmaf(f, v.w, acc.w);
+    }
+    const float inv = (Ls > 0.f) ? 1.f / Ls : 0.f;
+    uint2 pk;
+    pk.x = pack_bf16(acc.x * inv, acc.y * inv);
+    pk.y = pack_bf16(acc.z * inv, acc.w * inv);
+    *(uint2 *)(out + (long)pair * 128 + lane * 4) = pk;
+    if (lse && lane == 0)
+        lse[pair] = (Ls > 0.f) ? (M + __log2f(Ls)) * 0.6931471805599453f : -INFINITY;
+}
+
+cudaError_t launch_attn_decode(const inkling_decode_params &p, int splits, void *workspace,
+                               const CUtensorMap &tm_k, const CUtensorMap &tm_v,
+                               cudaStream_t stream) {
+    DecodeArgs a;
+    a.q = (const uint16_t *)p.q;
+    a.block_table = p.block_table;
+    a.seq_lens = p.seq_lens;
+    a.bias = p.bias;
+    a.out = (uint16_t *)p.out;
+    a.lse = p.lse;
+    const long pairs = (long)p.num_seqs * p.num_q_heads;
+    a.part_o = (float *)workspace;
+    a.part_ml = splits > 1 ? (float *)workspace + pairs * splits * 128 : nullptr;
+    a.status = p.status;
+    a.S = p.num_seqs;
+    a.Hq = p.num_q_heads;
+    a.Hkv = p.num_kv_heads;
+    a.G = p.num_q_heads / p.num_kv_heads;
+    a.max_blocks = p.max_blocks;
+    a.num_blocks = p.num_blocks;
+    a.window = p.window;
+    a.d_max = p.d_max;
+    a.splits = splits;
+    cudaError_t e0 = cudaFuncSetAttribute(decode_split_kernel,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
+    if (e0 != cudaSuccess) return e0;
+    const long grid = (long)p.num_seqs * p.num_kv_heads * splits;
+    decode_split_kernel<<<(unsigned)grid, 160, kDecSmem, stream>>>(tm_k, tm_v, a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || splits == 1) return e;
+    decode_combine_kernel<<<(unsigned)((pairs + 3) / 4), 128, 0, stream>>>(
+        a.part_o, a.part_ml, a.out, a.lse, (int)pairs, splits);
+    return cudaGetLastError();
+}
+
+}  // namespace inkling

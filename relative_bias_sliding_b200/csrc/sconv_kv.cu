@@ -1,0 +1,88 @@
+// sconv_kv.cu — decode-side sconv append (vLLM Recipes "thinkingmachines/
+// Inkling", Overview, "Short convolution": window-4 sconv on keys and values,
+// its state managed like the KV cache of a sliding-window layer).
+//
+// One thread owns 8 consecutive channels of one sequence's keys or values:
+// it reads the 3 raw history tokens from the state, convolves each new token,
+// writes the bf16 result to the token's slot in the paged cache
+// (block_table[s, pos/128], slot pos%128) and stores the last 3 raw tokens
+// back as the new state.  Memory-bound: 16-byte loads and stores, one pass.
+#include "common.cuh"
+
+namespace inkling {
+
+__global__ void __launch_bounds__(128)
+sconv_kv_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new,
+                const float4 *__restrict__ w_k, const float4 *__restrict__ w_v,
+                uint4 *__restrict__ k_state, uint4 *__restrict__ v_state,
+                uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache,
+                const int32_t *__restrict__ block_table, const int32_t *__restrict__ seq_lens,
+                int32_t *status, int S, int n_new, int Hkv, int max_blocks, int num_blocks) {
+    const int chunks = Hkv * 16;  // 8-channel chunks per token (C = Hkv*128)
+    const long gid = (long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= (long)S * 2 * chunks) return;
+    const int chunk = (int)(gid % chunks);
+    const int which = (int)((gid / chunks) & 1);  // 0 = keys, 1 = values
+    const int s = (int)(gid / (2 * chunks));
+
+    const uint4 *xin = which ? v_new : k_new;
+    const float4 *wt = which ? w_v : w_k;
+    uint4 *state = which ? v_state : k_state;
+    uint4 *cache = which ? v_cache : k_cache;
+
+    const int L = seq_lens[s];
+    if (L < n_new || L > max_blocks * 128) {
+        report_status(status, INKLING_STATUS_BAD_LENGTH);
+        return;
+    }
+    float w[8][4];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const float4 t = wt[chunk * 8 + e];
+        w[e][0] = t.x; w[e][1] = t.y; w[e][2] = t.z; w[e][3] = t.w;
+    }
+    // state [S, 3, C] bf16 = per token `chunks` uint4
+    float h3[8], h2[8], h1[8];
+    uint4 r3 = state[((long)s * 3 + 0) * chunks + chunk];
+    uint4 r2 = state[((long)s * 3 + 1) * chunks + chunk];
+    uint4 r1 = state[((long)s * 3 + 2) * chunks + chunk];
+    unpack8(r3, h3);
+    unpack8(r2, h2);
+    unpack8(r1, h1);
+
+    const int kvh = chunk >> 4, e16 = chunk & 15;  // kv head, 16-byte column in the row
+    for (int t = 0; t < n_new; ++t) {
+        const uint4 raw = xin[((long)s * n_new + t) * chunks + chunk];
+        float x[8];
+        unpack8(raw, x);
+        const uint4 y = sconv8(w, h3, h2, h1, x);
+        const int pos = L - n_new + t;
+        const int blk = block_table[(long)s * max_blocks + (pos >> 7)];
+        if (blk < 0 || blk >= num_blocks) {
+            report_status(status, INKLING_STATUS_BAD_BLOCK);
+        } else {
+            cache[(((long)blk * Hkv + kvh) * 128 + (pos & 127)) * 16 + e16] = y;
+        }
+        r3 = r2; r2 = r1; r1 = raw;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) { h3[e] = h2[e]; h2[e] = h1[e]; h1[e] = x[e]; }
+    }
+    state[((long)s * 3 + 0) * chunks + chunk] = r3;
+    state[((long)s * 3 + 1) * chunks + chunk] = r2;
+    state[((long)s * 3 + 2) * chunks + chunk] = r1;
+}
+
+cudaError_t launch_sconv_kv(const inkling_sconv_params &p, cudaStream_t stream) {
+    const long threads = (long)p.num_seqs * 2 * p.num_kv_heads * 16;
+    if (threads == 0) return cudaSuccess;
+    const int block = 128;
+    const long grid = (threads + block - 1) / block;
+    sconv_kv_kernel<<<(unsigned)grid, block, 0, stream>>>(
+        (const uint4 *)p.k_new, (const uint4 *)p.v_new, (const float4 *)p.w_k,
+        (const float4 *)p.w_v, (uint4 *)p.k_state, (uint4 *)p.v_state, (uint4 *)p.k_cache,
+        (uint4 *)p.v_cache, p.block_table, p.seq_lens, p.status, p.num_seqs, p.n_new,
+        p.num_kv_heads, p.max_blocks, p.num_blocks);
+    return cudaGetLastError();
+}
+
+}  // namespace inkling

@@ -1,0 +1,113 @@
+"""The C-ABI library loads, exports every entry point include/inkling.h
+declares, its parameter structs match the ctypes mirrors byte for byte, and
+host-side validation rejects bad arguments before touching a device (CPU)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from relative_bias_sliding_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "inkling.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(inkling_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert set(names) == set(binding.EXPORTED)
+    out = subprocess.run(["nm", "-D", "--defined-only", binding.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (inkling_\w+)", out))
+    for n in names:
+        assert n in exported, n
+        assert hasattr(lib, n)
+
+
+def test_struct_layouts_match_header(tmp_path):
+    src = tmp_path / "sizes.c"
+    src.write_text(f"""
+#include <stddef.h>
+#include <stdio.h>
+#include "{HEADER}"
+#define F(S, m) printf(#S " " #m " %zu\\n", offsetof(S, m));
+int main(void) {{
+  printf("sconv %zu\\nprefill %zu\\ndecode %zu\\n", sizeof(inkling_sconv_params),
+         sizeof(inkling_prefill_params), sizeof(inkling_decode_params));
+  F(inkling_sconv_params, num_blocks) F(inkling_prefill_params, d_max)
+  F(inkling_decode_params, num_splits) F(inkling_decode_params, status)
+  return 0;
+}}""")
+    exe = tmp_path / "sizes"
+    subprocess.run(["gcc", str(src), "-o", str(exe)], check=True)
+    out = dict(l.rsplit(" ", 1) for l in subprocess.run([str(exe)], capture_output=True,
+                                                         text=True).stdout.splitlines())
+    assert int(out["sconv"]) == ctypes.sizeof(binding.SconvParams)
+    assert int(out["prefill"]) == ctypes.sizeof(binding.PrefillParams)
+    assert int(out["decode"]) == ctypes.sizeof(binding.DecodeParams)
+    assert int(out["inkling_sconv_params num_blocks"]) == binding.SconvParams.num_blocks.offset
+    assert int(out["inkling_prefill_params d_max"]) == binding.PrefillParams.d_max.offset
+    assert int(out["inkling_decode_params num_splits"]) == binding.DecodeParams.num_splits.offset
+    assert int(out["inkling_decode_params status"]) == binding.DecodeParams.status.offset
+
+
+def test_workspace_bytes(lib):
+    f = lib.inkling_attn_decode_workspace_bytes
+    assert f(64, 64, 4) == 64 * 64 * 4 * 130 * 4
+    assert f(1, 64, 148) == 64 * 148 * 130 * 4
+    assert f(3, 8, 1) == 16
+    assert f(-1, 8, 2) == 0 and f(3, 0, 2) == 0 and f(3, 8, 0) == 0 and f(3, 8, 1025) == 0
+
+
+def test_host_validation_rejects_before_launch(lib):
+    # none of these reach the device: they fail argument checks first
+    p = binding.PrefillParams()
+    p.batch, p.seq_len, p.num_q_heads, p.num_kv_heads, p.head_dim = 1, 16, 8, 1, 64
+    assert lib.inkling_attn_prefill(ctypes.byref(p), None) == binding.INKLING_ERR_UNSUPPORTED
+    assert b"head_dim" in lib.inkling_last_error()
+    p.head_dim, p.num_q_heads, p.num_kv_heads = 128, 6, 4
+    assert lib.inkling_attn_prefill(ctypes.byref(p), None) == binding.INKLING_ERR_INVALID
+    p.num_q_heads = 8
+    assert lib.inkling_attn_prefill(ctypes.byref(p), None) == binding.INKLING_ERR_INVALID  # NULLs
+    p.batch = 0
+    assert lib.inkling_attn_prefill(ctypes.byref(p), None) == binding.INKLING_OK  # empty: no-op
+    assert lib.inkling_attn_prefill(None, None) == binding.INKLING_ERR_INVALID
+
+    d = binding.DecodeParams()
+    d.num_seqs, d.num_q_heads, d.num_kv_heads, d.head_dim = 2, 64, 4, 128
+    d.max_blocks, d.num_blocks = 4, 8
+    assert lib.inkling_attn_decode(ctypes.byref(d), None, 0, None) == binding.INKLING_ERR_UNSUPPORTED
+    d.num_kv_heads = 8
+    assert lib.inkling_attn_decode(ctypes.byref(d), None, 0, None) == binding.INKLING_ERR_INVALID
+    d.num_splits = 2000
+    assert lib.inkling_attn_decode(ctypes.byref(d), None, 0, None) == binding.INKLING_ERR_INVALID
+
+    s = binding.SconvParams()
+    s.num_seqs, s.n_new, s.num_kv_heads, s.head_dim, s.max_blocks, s.num_blocks = 1, 65, 1, 128, 1, 1
+    assert lib.inkling_sconv_kv(ctypes.byref(s), None) == binding.INKLING_ERR_INVALID
+    s.n_new = 1
+    assert lib.inkling_sconv_kv(ctypes.byref(s), None) == binding.INKLING_ERR_INVALID  # NULLs
+
+
+def test_product_path_does_not_import_oracle():
+    # the binding, the build script and the kernels never reference the oracle
+    pkg = os.path.join(ROOT, "relative_bias_sliding_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f
+                assert "liboracle" not in text and "oracle.c" not in text, f

@@ -1,0 +1,154 @@
+"""tcgen05 prefill (fused sconv) on the GPU against the oracle, plus invariants."""
+import numpy as np
+import pytest
+import torch
+
+from conftest import assert_parity, need_gpu, u16
+import relative_bias_sliding_b200 as ink
+from relative_bias_sliding_b200.inputs import WORKLOADS, make_prefill, scaled
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(t, window, with_lse=True):
+    dev = {k: v.cuda() for k, v in t.items()}
+    B, T, Hq, _ = dev["q"].shape
+    lse = torch.empty((B, Hq, T), dtype=torch.float32, device="cuda") if with_lse else None
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = ink.attn_prefill(dev["q"], dev["k_raw"], dev["v_raw"], dev["w_k"], dev["w_v"],
+                           dev["bias"], window=window, lse=lse, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0, f"status {status.item()}"
+    return out, lse
+
+
+def _oracle_all(oracle_mod, t, window):
+    out, lse, _, _ = oracle_mod.prefill_rows(u16(t["q"]), u16(t["k_raw"]), u16(t["v_raw"]),
+                                             t["w_k"].numpy(), t["w_v"].numpy(),
+                                             t["bias"].numpy(), window, t["bias"].shape[1] - 1)
+    return out, lse
+
+
+def test_prefill_tiny_workload_all_rows(oracle_mod):
+    need_gpu()
+    spec = WORKLOADS["prefill_tiny_b1_t256"]
+    t = make_prefill(spec)
+    out, lse = _run(t, spec.window)
+    ref, ref_lse = _oracle_all(oracle_mod, t, spec.window)
+    assert_parity(out, ref, spec.name)
+    got_lse = lse.permute(0, 2, 1).cpu().numpy().reshape(-1)   # [B, T, Hq] order
+    np.testing.assert_allclose(got_lse, ref_lse, rtol=0, atol=2e-3)
+
+
+@pytest.mark.parametrize("B,T,Hq,Hkv,W,D_max", [
+    (1, 1, 8, 1, 0, 16),         # a single token
+    (1, 129, 8, 1, 0, 256),      # one row past a tile
+    (2, 300, 8, 2, 0, 64),       # ragged tail, GQA 4, clip inside the band
+    (1, 700, 4, 1, 100, 1000),   # window narrower than a tile
+    (1, 640, 8, 8, 128, 128),    # window exactly one tile, G = 1
+    (1, 1000, 16, 2, 300, 50),   # window + clip, ragged
+    (1, 520, 8, 1, 1, 8),        # window of one key (self only)
+    (3, 257, 8, 4, 256, 300),    # query block boundary + 1
+])
+def test_prefill_ragged_and_masks(oracle_mod, B, T, Hq, Hkv, W, D_max):
+    need_gpu()
+    spec = scaled(WORKLOADS["prefill_tiny_b1_t256"], B=B, T=T, Hq=Hq, Hkv=Hkv, window=W,
+                  D_max=D_max, seed=T + W)
+    t = make_prefill(spec)
+    out, _ = _run(t, W)
+    ref, _ = _oracle_all(oracle_mod, t, W)
+    assert_parity(out, ref, f"B{B} T{T} Hq{Hq} Hkv{Hkv} W{W} D{D_max}")
+
+
+def test_prefill_window_at_least_T_equals_full():
+    need_gpu()
+    spec = scaled(WORKLOADS["prefill_tiny_b1_t256"], T=600, Hq=8, Hkv=2, D_max=700, seed=5)
+    t = make_prefill(spec)
+    full, _ = _run(t, 0)
+    win, _ = _run(t, 600)
+    assert torch.equal(full, win)
+
+
+def test_prefill_empty_batch_is_noop():
+    need_gpu()
+    spec = scaled(WORKLOADS["prefill_tiny_b1_t256"], B=1, T=16)
+    t = make_prefill(spec)
+    dev = {k: v.cuda() for k, v in t.items()}
+    out = torch.full((0, 16, 8, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    ink.attn_prefill(dev["q"][:0], dev["k_raw"][:0], dev["v_raw"][:0], dev["w_k"], dev["w_v"],
+                     dev["bias"], out=out)
+    torch.cuda.synchronize()
+
+
+def test_prefill_last_row_equals_decode(oracle_mod):
+    """Prefill row T-1 equals decode at length T over the cache that
+    sconv_kv builds from the same raw keys and values (streaming continuity)."""
+    need_gpu()
+    T, Hq, Hkv, W, D = 1000, 16, 2, 300, 512
+    spec = scaled(WORKLOADS["prefill_tiny_b1_t256"], T=T, Hq=Hq, Hkv=Hkv, window=W, D_max=D,
+                  seed=3)
+    t = make_prefill(spec)
+    out, _ = _run(t, W)
+    dev = {k: v.cuda() for k, v in t.items()}
+    nb = (T + 127) // 128
+    kc = torch.zeros((nb + 2, Hkv, 128, 128), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    bt = torch.arange(2, nb + 2, dtype=torch.int32, device="cuda")[None]
+    ks = torch.zeros((1, 3, Hkv * 128), dtype=torch.bfloat16, device="cuda")
+    vs = torch.zeros_like(ks)
+    done = 0
+    while done < T:
+        n = min(64, T - done)
+        ink.sconv_kv(dev["k_raw"][:, done:done + n].contiguous(),
+                     dev["v_raw"][:, done:done + n].contiguous(), dev["w_k"], dev["w_v"], ks, vs,
+                     kc, vc, bt, torch.tensor([done + n], dtype=torch.int32, device="cuda"))
+        done += n
+    dec = ink.attn_decode(dev["q"][:, T - 1].contiguous(), kc, vc, bt,
+                          torch.tensor([T], dtype=torch.int32, device="cuda"), dev["bias"],
+                          window=W, num_splits=3)
+    torch.cuda.synchronize()
+    assert (dec.float() - out[:, T - 1].float()).abs().max().item() < 2e-2
+    rows = np.array([[0, h, T - 1] for h in range(Hq)], np.int32)
+    ref, _, _, _ = oracle_mod.prefill_rows(u16(t["q"]), u16(t["k_raw"]), u16(t["v_raw"]),
+                                           t["w_k"].numpy(), t["w_v"].numpy(), t["bias"].numpy(),
+                                           W, D, rows)
+    assert_parity(dec[0], ref, "decode vs oracle")
+
+
+def _sample_rows(spec, rng, per_head):
+    """Rows that exercise every mask case: first rows, the window edge, tile
+    and query-block boundaries, the last rows, and random rows."""
+    T, W = spec.T, spec.window
+    fixed = [0, 1, 127, 128, 255, 256, T - 1, T - 2, T - 129]
+    if W > 0:
+        fixed += [W - 1, W, W + 1, W + 127, W + 128]
+    fixed = [i for i in fixed if 0 <= i < T]
+    rows = []
+    for b in range(spec.B):
+        for h in range(spec.Hq):
+            pick = list(fixed) + list(rng.integers(0, T, size=per_head))
+            rows += [(b, h, i) for i in pick]
+    return np.array(rows, np.int32)
+
+
+@pytest.mark.parametrize("name,per_head", [("prefill_swa_b4_t8192", 4),
+                                           ("prefill_full_b1_t32768", 3)])
+def test_prefill_full_size_sampled_rows(oracle_mod, name, per_head):
+    """The benchmark workloads at full size, in the benchmark's launch
+    configuration; the oracle computes a sample of rows of every (batch, head)."""
+    need_gpu()
+    spec = WORKLOADS[name]
+    t = make_prefill(spec, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = ink.attn_prefill(t["q"], t["k_raw"], t["v_raw"], t["w_k"], t["w_v"], t["bias"],
+                           window=spec.window, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    rows = _sample_rows(spec, np.random.default_rng(0), per_head)
+    ref, _, _, _ = oracle_mod.prefill_rows(u16(t["q"]), u16(t["k_raw"]), u16(t["v_raw"]),
+                                           t["w_k"].cpu().numpy(), t["w_v"].cpu().numpy(),
+                                           t["bias"].cpu().numpy(), spec.window, spec.D_max,
+                                           rows)
+    r = torch.from_numpy(rows).long().cuda()
+    got = out[r[:, 0], r[:, 2], r[:, 1]].float().cpu().numpy()
+    assert_parity(got, ref, name)
