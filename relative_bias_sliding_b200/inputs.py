@@ -83,6 +83,12 @@ WORKLOADS = {
                                     1 << 20, 0.5, 4),
     "decode_full_1m_b8": DecodeSpec("decode_full_1m_b8", 8, 1 << 20, 1 << 20, 64, 8, 128, 0,
                                     1 << 20, 0.5, 4),
+    # smaller cuts of the same workloads for profiler captures (still larger
+    # than L2, a few GB on the device at most)
+    "prefill_swa_b1_t8192": PrefillSpec("prefill_swa_b1_t8192", 1, 8192, 64, 8, 128, 4096,
+                                        4096, 1.0, 1),
+    "decode_swa_s16": DecodeSpec("decode_swa_s16", 16, 1024, 32768, 64, 8, 128, 4096, 4096,
+                                 1.0, 3),
 }
 
 
