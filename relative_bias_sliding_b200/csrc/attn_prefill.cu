@@ -13,7 +13,7 @@
 // Warp roles (16 warps):
 //   0-3   softmax of query tile 0 (thread = one query row = one TMEM lane)
 //   4-7   softmax of query tile 1
-//   8-11  sconv transform: converts the raw key / value tile in place
+//   8-9   sconv of the key tile, 10-11 sconv of the value tile (in place)
 //   12    TMA producer (Q once; raw K, raw V and their 3-row history per tile)
 //   13    TMEM allocator and single-thread tcgen05.mma issuer
 //   14-15 idle
@@ -35,9 +35,11 @@ constexpr uint32_t SM_K = 65536;        // 2 stages x 32 KB
 constexpr uint32_t SM_V = 131072;       // 2 stages x 32 KB
 constexpr uint32_t SM_KH = 196608;      // 2 stages x 2 KB (8 history rows x 2 halves)
 constexpr uint32_t SM_VH = 200704;      // 2 stages x 2 KB
-constexpr uint32_t SM_W = 204800;       // w_k (2 KB) + w_v (2 KB) of this kv head
-constexpr uint32_t SM_BAR = 208896;     // mbarriers, tmem base, abort flag, verdict
-constexpr int kPrefillSmem = 208896 + 512 + 1024;
+constexpr uint32_t SM_BIAS = 204800;    // 2 softmax groups x 2 buffers x 4 copies x 264 fp32
+constexpr int kBiasCopy = 264;          // floats per shifted copy (== 8 mod 32: conflict-free)
+constexpr int kBiasBuf = 4 * kBiasCopy;
+constexpr uint32_t SM_BAR = SM_BIAS + 2 * 2 * kBiasBuf * 4;  // mbarriers, tmem base, flags
+constexpr int kPrefillSmem = SM_BAR + 512 + 1024;
 
 enum {
     B_QFULL = 0,
@@ -62,52 +64,63 @@ struct PrefillArgs {
     int B, T, Hq, Hkv, window, d_max, nqb;
 };
 
-// Register split per warpgroup: 2 x 128 softmax threads at 184, 128 sconv
-// threads at 96, 128 producer/MMA/idle threads at 48: 47104 + 12288 + 6144 =
+// Register split per warpgroup: 2 x 128 softmax threads at 176, 128 sconv
+// threads at 112, 128 producer/MMA/idle threads at 48: 45056 + 14336 + 6144 =
 // 65536 = 512 threads x the 128 registers the kernel launches with (ptxas
 // reports 128), so the increase never waits on registers that do not exist.
-INK_DEV void setmaxnreg_inc184() { asm volatile("setmaxnreg.inc.sync.aligned.u32 184;"); }
-INK_DEV void setmaxnreg_dec96() { asm volatile("setmaxnreg.dec.sync.aligned.u32 96;"); }
+INK_DEV void setmaxnreg_inc176() { asm volatile("setmaxnreg.inc.sync.aligned.u32 176;"); }
+INK_DEV void setmaxnreg_dec112() { asm volatile("setmaxnreg.dec.sync.aligned.u32 112;"); }
 INK_DEV void setmaxnreg_dec48() { asm volatile("setmaxnreg.dec.sync.aligned.u32 48;"); }
 
 // Convert one raw 128-row key or value tile (TMA layout: two 64-column halves
-// of 128 rows x 128 bytes, 128-byte swizzle) into its sconv output, in place.
-// Thread u owns 16-byte column c = u % 16 (8 channels) and rows 16g..16g+15,
-// g = u / 16; the 3 rows before its first row come from the tile itself, or
-// for g = 0 from the 8-row history box loaded with the tile.
-INK_DEV void sconv_tile_inplace(uint32_t tile, uint32_t hist, const float *wsm, int u) {
-    const int c = u & 15, g = u >> 4;
+// of 128 rows x 128 bytes, 128-byte swizzle) into its sconv output, in place,
+// with 64 threads.  Thread v owns 16-byte column c = v % 16 (8 channels) and
+// rows 32g..32g+31, g = v / 16; the 3 rows before its first row come from the
+// tile itself, or for g = 0 from the 8-row history box loaded with the tile.
+// w[tap][pair] holds the taps of channel pairs (2p, 2p+1) of this column.
+INK_DEV void sconv_tile_group(uint32_t tile, uint32_t hist, const f32x2 (&w)[4][4], int v,
+                              int bar_id) {
+    const int c = v & 15, g = v >> 4;
     const int half = c >> 3, cc = c & 7;
-    float w[8][4];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        const float4 t4 = *(const float4 *)(wsm + (c * 8 + e) * 4);
-        w[e][0] = t4.x; w[e][1] = t4.y; w[e][2] = t4.z; w[e][3] = t4.w;
-    }
-    float h3[8], h2[8], h1[8];
+    const uint32_t tb = tile + half * 16384;
+    f32x2 h3[4], h2[4], h1[4];
+    auto load = [&](uint32_t base, int r, f32x2(&dst)[4]) {
+        const uint4 q = lds128(base + r * 128 + ((cc ^ (r & 7)) << 4));
+        dst[0] = bf2_to_f2(q.x);
+        dst[1] = bf2_to_f2(q.y);
+        dst[2] = bf2_to_f2(q.z);
+        dst[3] = bf2_to_f2(q.w);
+    };
     if (g == 0) {
         const uint32_t hb = hist + half * 1024;
-        unpack8(lds128(hb + 5 * 128 + ((cc ^ 5) << 4)), h3);
-        unpack8(lds128(hb + 6 * 128 + ((cc ^ 6) << 4)), h2);
-        unpack8(lds128(hb + 7 * 128 + ((cc ^ 7) << 4)), h1);
+        load(hb, 5, h3);
+        load(hb, 6, h2);
+        load(hb, 7, h1);
     } else {
-        const uint32_t tb = tile + half * 16384;
-        const int r = 16 * g;
-        unpack8(lds128(tb + (r - 3) * 128 + ((cc ^ ((r - 3) & 7)) << 4)), h3);
-        unpack8(lds128(tb + (r - 2) * 128 + ((cc ^ ((r - 2) & 7)) << 4)), h2);
-        unpack8(lds128(tb + (r - 1) * 128 + ((cc ^ ((r - 1) & 7)) << 4)), h1);
+        load(tb, 32 * g - 3, h3);
+        load(tb, 32 * g - 2, h2);
+        load(tb, 32 * g - 1, h1);
     }
-    named_bar_sync(1, 128);  // every history row read before any row is overwritten
-    const uint32_t tb = tile + half * 16384;
+    named_bar_sync(bar_id, 64);  // every history row read before any row is overwritten
 #pragma unroll 4
-    for (int i = 0; i < 16; ++i) {
-        const int r = 16 * g + i;
+    for (int i = 0; i < 32; ++i) {
+        const int r = 32 * g + i;
         const uint32_t addr = tb + r * 128 + ((cc ^ (r & 7)) << 4);
-        float x[8];
-        unpack8(lds128(addr), x);
-        sts128(addr, sconv8(w, h3, h2, h1, x));
+        f32x2 x[4];
+        load(tb, r, x);
+        uint32_t o[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) { h3[e] = h2[e]; h2[e] = h1[e]; h1[e] = x[e]; }
+        for (int p = 0; p < 4; ++p) {
+            // same order as the decode append: w3*x[t-3], +w2*x[t-2], +w1*x[t-1], +w0*x[t]
+            f32x2 acc = fmul2(w[3][p], h3[p]);
+            acc = ffma2(w[2][p], h2[p], acc);
+            acc = ffma2(w[1][p], h1[p], acc);
+            acc = ffma2(w[0][p], x[p], acc);
+            o[p] = f2_to_bf2(acc);
+        }
+        sts128(addr, make_uint4(o[0], o[1], o[2], o[3]));
+#pragma unroll
+        for (int p = 0; p < 4; ++p) { h3[p] = h2[p]; h2[p] = h1[p]; h1[p] = x[p]; }
     }
 }
 
@@ -123,7 +136,6 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
     uint64_t *bar = (uint64_t *)(smem + SM_BAR);
     uint32_t *tmem_slot = (uint32_t *)(bar + B_COUNT);
     volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
-    float *w_sm = (float *)(smem + SM_W);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -149,20 +161,18 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
 
     // ---- setup
     if (threadIdx.x == 0) {
-        for (int i = 0; i < B_COUNT; ++i) mbar_init(&bar[i], (i == B_PFULL || i == B_PFULL + 1) ? 128 : 1);
+        for (int i = 0; i < B_COUNT; ++i) {
+            uint32_t cnt = 1;
+            if (i == B_PFULL || i == B_PFULL + 1) cnt = 128;
+            if (i == B_KREADY || i == B_KREADY + 1 || i == B_VREADY || i == B_VREADY + 1) cnt = 64;
+            mbar_init(&bar[i], cnt);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 13) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
-    }
-    if (warp >= 8 && warp < 12) {
-        const int u = threadIdx.x - 256;
-        const float4 *wk = (const float4 *)(a.w_k + (long)kvh * 512);
-        const float4 *wv = (const float4 *)(a.w_v + (long)kvh * 512);
-        ((float4 *)w_sm)[u] = wk[u];
-        ((float4 *)(w_sm + 512))[u] = wv[u];
     }
     tc_fence_before();
     __syncthreads();
@@ -171,7 +181,7 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
 
     if (warp < 8) {
         // ================================================== softmax (2 WGs) ==
-        setmaxnreg_inc184();
+        setmaxnreg_inc176();
         const int t = warp >> 2;
         const int u = threadIdx.x & 127;
         if (ok[t]) {
@@ -184,13 +194,33 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
             const float *bias_h = a.bias + (long)h * (a.d_max + 1);
             const int W = a.window, Dm = a.d_max, T = a.T;
             float m_ref = -INFINITY, l = 0.f;
+            float *bias_sm = (float *)(smem + SM_BIAS) + t * 2 * kBiasBuf;
+            const int o_rd = 127 - u, sh = o_rd & 3;  // this row's start in the staged diagonal
+            bool dead = false;
             int k = 0;
-            bool aborted = false;
             for (int n = lo[t]; n <= hi[t]; ++n, ++k) {
-                if (!mbar_wait_warp(&bar[B_SFULL + t], k & 1, abort_flag, a.status)) {
-                    aborted = true;
-                    break;
+                const int j0 = n * 128;
+                // Stage the bias diagonal of this (query tile, key tile) pair:
+                // R[q] = bias[h, clamp(top - q, 0, d_max)], q = 0..254, top = r0 - j0 + 127,
+                // as 4 copies shifted by 0..3 floats so that row u reads R[127-u+c],
+                // c = 0..127, with aligned 16-byte loads.  Double-buffered by tile parity.
+                float *bb = bias_sm + (k & 1) * kBiasBuf;
+                {
+                    const int top = r0[t] - j0 + 127;
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int q = 2 * u + e;
+                        if (q < 255) {
+                            const float bv = __ldg(bias_h + min(max(top - q, 0), Dm));
+#pragma unroll
+                            for (int s4 = 0; s4 < 4; ++s4)
+                                if (q >= s4) bb[s4 * kBiasCopy + q - s4] = bv;
+                        }
+                    }
                 }
+                named_bar_sync(3 + t, 128);
+                if (!dead) dead = !mbar_wait_warp(&bar[B_SFULL + t], k & 1, abort_flag, a.status);
+                if (dead) continue;  // keep stepping through the group barrier
                 tc_fence_after();
                 uint32_t sr[128];
                 tmem_ld32(s_col + 0, sr + 0);
@@ -198,35 +228,48 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                 tmem_ld32(s_col + 64, sr + 64);
                 tmem_ld32(s_col + 96, sr + 96);
                 tmem_wait_ld();
+                const float4 *rp = (const float4 *)(bb + sh * kBiasCopy + (o_rd - sh));
                 float x[128];
-                const int j0 = n * 128;
                 const int dist0 = i - j0;  // distance of key j0 + c is dist0 - c
                 const bool full = (dist0 - 127 >= 0) && (W <= 0 || dist0 < W) && (j0 + 127 < T);
-                float mx = -INFINITY;
-                if (full && dist0 <= Dm) {
-                    const float *bp = bias_h + dist0;
+                if (full) {
+                    const f32x2 sc2 = pk2(scale, scale);
 #pragma unroll
-                    for (int c = 0; c < 128; ++c) {
-                        x[c] = fmaf(__uint_as_float(sr[c]), scale, __ldg(bp - c));
-                        mx = fmaxf(mx, x[c]);
-                    }
-                } else if (full && dist0 - 127 >= Dm) {
-                    const float bc = __ldg(bias_h + Dm);
-#pragma unroll
-                    for (int c = 0; c < 128; ++c) {
-                        x[c] = fmaf(__uint_as_float(sr[c]), scale, bc);
-                        mx = fmaxf(mx, x[c]);
+                    for (int c4 = 0; c4 < 32; ++c4) {
+                        const float4 b4 = rp[c4];
+                        const f32x2 xa = ffma2(pk2(__uint_as_float(sr[4 * c4]),
+                                                   __uint_as_float(sr[4 * c4 + 1])),
+                                               sc2, pk2(b4.x, b4.y));
+                        const f32x2 xb = ffma2(pk2(__uint_as_float(sr[4 * c4 + 2]),
+                                                   __uint_as_float(sr[4 * c4 + 3])),
+                                               sc2, pk2(b4.z, b4.w));
+                        upk2(xa, x[4 * c4], x[4 * c4 + 1]);
+                        upk2(xb, x[4 * c4 + 2], x[4 * c4 + 3]);
                     }
                 } else {
 #pragma unroll
-                    for (int c = 0; c < 128; ++c) {
-                        const int dist = dist0 - c;
-                        const bool allowed = dist >= 0 && (W <= 0 || dist < W) && (j0 + c < T);
-                        const float bv = allowed ? __ldg(bias_h + min(dist, Dm)) : 0.f;
-                        x[c] = allowed ? fmaf(__uint_as_float(sr[c]), scale, bv) : -INFINITY;
-                        mx = fmaxf(mx, x[c]);
+                    for (int c4 = 0; c4 < 32; ++c4) {
+                        const float4 b4 = rp[c4];
+                        const float bq[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int c = 4 * c4 + e;
+                            const int dist = dist0 - c;
+                            const bool allowed = dist >= 0 && (W <= 0 || dist < W) && (j0 + c < T);
+                            x[c] = allowed ? fmaf(__uint_as_float(sr[c]), scale, bq[e]) : -INFINITY;
+                        }
                     }
                 }
+                // row max: 8 independent chains of 3-input max
+                float m8[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) m8[q] = fmaxf(x[2 * q], x[2 * q + 1]);
+#pragma unroll
+                for (int c = 16; c < 128; c += 16)
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) m8[q] = max3f(m8[q], x[c + 2 * q], x[c + 2 * q + 1]);
+                const float mx = fmaxf(max3f(m8[0], m8[1], m8[2]),
+                                       max3f(max3f(m8[3], m8[4], m8[5]), m8[6], m8[7]));
                 // lazy rescale: move the reference only when the max grows by > tau
                 const bool grow = mx > m_ref + kTau;
                 float alpha = 1.f;
@@ -237,16 +280,24 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                 }
                 const float mneg = (m_ref == -INFINITY) ? 0.f : -m_ref * kLog2e;
                 {
+                    const f32x2 l2e2 = pk2(kLog2e, kLog2e), mneg2 = pk2(mneg, mneg);
+                    f32x2 acc[4] = {0ull, 0ull, 0ull, 0ull};
                     uint32_t pk[64];
 #pragma unroll
                     for (int c = 0; c < 64; ++c) {
-                        const float p0 = ex2(fmaf(x[2 * c], kLog2e, mneg));
-                        const float p1 = ex2(fmaf(x[2 * c + 1], kLog2e, mneg));
-                        l += p0 + p1;
+                        const f32x2 tt = ffma2(pk2(x[2 * c], x[2 * c + 1]), l2e2, mneg2);
+                        float t0, t1;
+                        upk2(tt, t0, t1);
+                        const float p0 = ex2(t0), p1 = ex2(t1);
+                        acc[c & 3] = fadd2(acc[c & 3], pk2(p0, p1));
                         pk[c] = pack_bf16(p0, p1);
                     }
                     tmem_st32(s_col + 0, pk + 0);
                     tmem_st32(s_col + 32, pk + 32);
+                    const f32x2 s01 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+                    float la, lb;
+                    upk2(s01, la, lb);
+                    l += la + lb;
                 }
                 // O rescale after P is out of registers (keeps the peak low); the
                 // P.V MMA of this tile is issued only after p_full
@@ -266,6 +317,7 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                 tc_fence_before();
                 mbar_arrive(&bar[B_PFULL + t]);
             }
+            const bool aborted = dead;
             // epilogue: O / l -> bf16
             if (!aborted && mbar_wait_warp(&bar[B_ODONE + t], 0, abort_flag, a.status)) {
                 tc_fence_after();
@@ -298,33 +350,36 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
     } else if (warp < 12) {
         // ============================================ sconv transform (WG2) ==
-        setmaxnreg_dec96();
-        const int u = threadIdx.x - 256;
-        volatile int *verdict = abort_flag + 1;
-        // one thread waits (bounded); the whole group learns the verdict at a
-        // named barrier, so no warp can be left alone inside a barrier
-        auto group_wait = [&](uint64_t *br, uint32_t parity) {
-            if (u == 0) *verdict = mbar_wait(br, parity, abort_flag, a.status) ? 1 : 0;
-            named_bar_sync(1, 128);
-            const bool good = *verdict != 0;
-            if (good) (void)mbar_try_wait(br, parity);
-            named_bar_sync(1, 128);  // verdict read by all before it is rewritten
-            return good;
-        };
+        setmaxnreg_dec112();
+        const bool is_v = warp >= 10;
+        const int v = threadIdx.x - (is_v ? 320 : 256);
+        const int bar_id = is_v ? 2 : 1;
+        // taps of this thread's 8 channels, as channel pairs, held for the whole block
+        f32x2 w[4][4];
+        {
+            const float *wg = (is_v ? a.w_v : a.w_k) + ((long)kvh * 128 + 8 * (v & 15)) * 4;
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+#pragma unroll
+                for (int tap = 0; tap < 4; ++tap)
+                    w[tap][p] = pk2(__ldg(wg + (2 * p) * 4 + tap), __ldg(wg + (2 * p + 1) * 4 + tap));
+        }
+        uint64_t *raw_full = &bar[is_v ? B_VRAW : B_KRAW];
+        uint64_t *ready = &bar[is_v ? B_VREADY : B_KREADY];
+        const uint32_t tiles = sb + (is_v ? SM_V : SM_K);
+        const uint32_t hists = sb + (is_v ? SM_VH : SM_KH);
+        bool dead = false;
         int it = 0;
         for (int n = ulo; n <= uhi; ++n, ++it) {
             const int st = it & 1;
-            const uint32_t ph = (it >> 1) & 1;
-            if (!group_wait(&bar[B_KRAW + st], ph)) break;
-            sconv_tile_inplace(sb + SM_K + st * 32768, sb + SM_KH + st * 2048, w_sm, u);
+            if (!dead) dead = !mbar_wait(&raw_full[st], (it >> 1) & 1, abort_flag, a.status);
+            if (dead) {
+                named_bar_sync(bar_id, 64);  // keep the group's barrier count matched
+                continue;
+            }
+            sconv_tile_group(tiles + st * 32768, hists + st * 2048, w, v, bar_id);
             fence_proxy_async_smem();
-            named_bar_sync(1, 128);
-            if (u == 0) mbar_arrive(&bar[B_KREADY + st]);
-            if (!group_wait(&bar[B_VRAW + st], ph)) break;
-            sconv_tile_inplace(sb + SM_V + st * 32768, sb + SM_VH + st * 2048, w_sm + 512, u);
-            fence_proxy_async_smem();
-            named_bar_sync(1, 128);
-            if (u == 0) mbar_arrive(&bar[B_VREADY + st]);
+            mbar_arrive(&ready[st]);
         }
     } else {
         setmaxnreg_dec48();

@@ -241,6 +241,47 @@ INK_DEV float ex2(float x) {
     return y;
 }
 
+// ---- packed fp32 pairs (two independent IEEE round-to-nearest operations
+// per instruction; each lane gives the same bits as the scalar operation)
+typedef unsigned long long f32x2;
+INK_DEV f32x2 pk2(float lo, float hi) {
+    f32x2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+INK_DEV void upk2(f32x2 v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+INK_DEV f32x2 ffma2(f32x2 a, f32x2 b, f32x2 c) {
+    f32x2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+INK_DEV f32x2 fmul2(f32x2 a, f32x2 b) {
+    f32x2 d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+INK_DEV f32x2 fadd2(f32x2 a, f32x2 b) {
+    f32x2 d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+INK_DEV float max3f(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+// bf16x2 word -> fp32 pair (element 0 = low half)
+INK_DEV f32x2 bf2_to_f2(uint32_t w) {
+    return pk2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+INK_DEV uint32_t f2_to_bf2(f32x2 v) {
+    float lo, hi;
+    upk2(v, lo, hi);
+    return pack_bf16(lo, hi);
+}
+
 INK_DEV uint4 lds128(uint32_t addr) {
     uint4 v;
     asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
