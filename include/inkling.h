@@ -24,7 +24,7 @@
  *  - Every pointer named "device" must point to device memory of the current
  *    CUDA device and be 16-byte aligned.  The caller owns all memory; the
  *    library allocates nothing and keeps no state except a per-thread error
- *    message.
+ *    message (and the scratch array of inkling_attn_decode_static).
  *  - Calls are asynchronous on `stream` (NULL = legacy default stream) and
  *    never synchronise.  Kernel faults surface at the caller's next
  *    synchronisation, as with any CUDA launch.
@@ -185,6 +185,30 @@ int32_t inkling_attn_decode_num_splits(const inkling_decode_params *p);
  * aligned, contents need no initialisation; not used when the split count is 1. */
 inkling_status inkling_attn_decode(const inkling_decode_params *p, void *workspace,
                                    size_t workspace_bytes, inkling_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * inkling_attn_decode_static — inkling_attn_decode with no caller workspace.
+ *
+ * The pages have no counterpart to this call.  It serves callers that can
+ * hand the library only their inputs and outputs and cannot obtain device
+ * memory for a workspace: code running under an allocator that owns the whole
+ * device and forbids other allocations, or a latency-critical decode loop in
+ * which an allocation (which may synchronise the device) is not acceptable.
+ *
+ * Same arguments and results as inkling_attn_decode.  The split partials go
+ * to an 8 MiB array that the library holds in device memory on every GPU
+ * that loads it, until the process exits; no allocation routine is called.
+ *  - The first call on a device asks the runtime for that array's address on
+ *    the current device; make that first call before any stream capture.
+ *  - With num_splits = 0 the split count is lowered, if needed, until the
+ *    partials fit (one split needs none).  An explicit num_splits whose
+ *    partials exceed 8 MiB returns INKLING_ERR_INVALID and launches nothing.
+ *  - All calls share the array and it keeps the last call's contents.  Every
+ *    partial a call reads is written earlier by the same call, so nothing
+ *    needs clearing, but calls that overlap on the GPU (e.g. on two streams
+ *    at once, on one device) race with each other: serialise them.
+ * -------------------------------------------------------------------------- */
+inkling_status inkling_attn_decode_static(const inkling_decode_params *p, inkling_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -8,6 +8,7 @@ marshals torch tensors into it and ``inputs`` draws seeded synthetic inputs.
 """
 from .binding import (  # noqa: F401
     attn_decode,
+    attn_decode_static,
     attn_prefill,
     decode_num_splits,
     decode_workspace_bytes,
@@ -15,5 +16,5 @@ from .binding import (  # noqa: F401
     sconv_kv,
 )
 
-__all__ = ["attn_prefill", "attn_decode", "sconv_kv", "decode_num_splits",
+__all__ = ["attn_prefill", "attn_decode", "attn_decode_static", "sconv_kv", "decode_num_splits",
            "decode_workspace_bytes", "load_library"]

@@ -30,6 +30,7 @@ EXPORTED = (
     "inkling_attn_decode_workspace_bytes",
     "inkling_attn_decode_num_splits",
     "inkling_attn_decode",
+    "inkling_attn_decode_static",
 )
 
 _P = ctypes.c_void_p
@@ -89,6 +90,8 @@ def load_library(path: str = LIB_PATH):
         lib.inkling_attn_decode_num_splits.restype = _I
         lib.inkling_attn_decode.argtypes = [ctypes.POINTER(DecodeParams), _P, ctypes.c_size_t, _P]
         lib.inkling_attn_decode.restype = ctypes.c_int
+        lib.inkling_attn_decode_static.argtypes = [ctypes.POINTER(DecodeParams), _P]
+        lib.inkling_attn_decode_static.restype = ctypes.c_int
         _lib = lib
         return lib
 
@@ -246,4 +249,17 @@ def attn_decode(q, k_cache, v_cache, block_table, seq_lens, bias, window=0, out=
     _dev(workspace, torch.uint8, "workspace")
     _check(lib.inkling_attn_decode(ctypes.byref(p), _ptr(workspace), workspace.numel(),
                                    _stream(stream)))
+    return out
+
+
+def attn_decode_static(q, k_cache, v_cache, block_table, seq_lens, bias, window=0, out=None,
+                       lse=None, num_splits=0, status=None, stream=None):
+    """Single-token paged decode that uses the library's own 8 MiB scratch for
+    the split partials instead of a workspace (for callers that cannot
+    allocate).  Calls must not overlap on the GPU; returns ``out``."""
+    if out is None:
+        out = torch.empty_like(q)
+    p = _decode_params(q, k_cache, v_cache, block_table, seq_lens, bias, window, out, lse, status,
+                       num_splits)
+    _check(load_library().inkling_attn_decode_static(ctypes.byref(p), _stream(stream)))
     return out

@@ -15,6 +15,7 @@ cudaError_t launch_attn_prefill(const inkling_prefill_params &p, const CUtensorM
 cudaError_t launch_attn_decode(const inkling_decode_params &p, int splits, void *workspace,
                                const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                                cudaStream_t stream);
+cudaError_t decode_static_scratch(void **ptr, size_t *bytes);
 }  // namespace inkling
 
 using namespace inkling;
@@ -232,6 +233,9 @@ int32_t inkling_attn_decode_num_splits(const inkling_decode_params *p) {
     return decode_splits(*p, sms);
 }
 
+static inkling_status decode_with(const inkling_decode_params *p, int splits, void *workspace,
+                                  size_t workspace_bytes, inkling_stream_t stream);
+
 inkling_status inkling_attn_decode(const inkling_decode_params *p, void *workspace,
                                    size_t workspace_bytes, inkling_stream_t stream) {
     g_err[0] = 0;
@@ -240,7 +244,39 @@ inkling_status inkling_attn_decode(const inkling_decode_params *p, void *workspa
     if (p->num_seqs == 0) return INKLING_OK;
     int sms = 0;
     if ((st = check_device(&sms)) != INKLING_OK) return st;
-    const int splits = decode_splits(*p, sms);
+    return decode_with(p, decode_splits(*p, sms), workspace, workspace_bytes, stream);
+}
+
+inkling_status inkling_attn_decode_static(const inkling_decode_params *p, inkling_stream_t stream) {
+    g_err[0] = 0;
+    inkling_status st = validate_decode(p);
+    if (st != INKLING_OK) return st;
+    if (p->num_seqs == 0) return INKLING_OK;
+    int sms = 0;
+    if ((st = check_device(&sms)) != INKLING_OK) return st;
+    void *scratch = nullptr;
+    size_t cap = 0;
+    cudaError_t e = decode_static_scratch(&scratch, &cap);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the decode scratch");
+    int splits = decode_splits(*p, sms);
+    if (inkling_attn_decode_workspace_bytes(p->num_seqs, p->num_q_heads, splits) > cap) {
+        if (p->num_splits > 0)
+            return fail(INKLING_ERR_INVALID,
+                        "num_splits %d needs %zu bytes of partials; the static scratch holds %zu "
+                        "(use fewer splits, or inkling_attn_decode with a workspace)",
+                        splits, inkling_attn_decode_workspace_bytes(p->num_seqs, p->num_q_heads, splits),
+                        cap);
+        // automatic split count: the largest that fits (1 needs no scratch)
+        while (splits > 1 &&
+               inkling_attn_decode_workspace_bytes(p->num_seqs, p->num_q_heads, splits) > cap)
+            --splits;
+    }
+    return decode_with(p, splits, scratch, cap, stream);
+}
+
+static inkling_status decode_with(const inkling_decode_params *p, int splits, void *workspace,
+                                  size_t workspace_bytes, inkling_stream_t stream) {
+    inkling_status st;
     if (splits > 1) {
         const size_t need = inkling_attn_decode_workspace_bytes(p->num_seqs, p->num_q_heads, splits);
         if (!workspace || workspace_bytes < need)

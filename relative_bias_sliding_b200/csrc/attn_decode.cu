@@ -20,6 +20,8 @@
 //  * the 4 warps merge through shared memory; with one split the block writes
 //    the bf16 output, otherwise an unnormalised partial (m, l, O) that
 //    decode_combine_kernel merges.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace inkling {
@@ -379,6 +381,35 @@ cudaError_t launch_attn_decode(const inkling_decode_params &p, int splits, void 
     decode_combine_kernel<<<(unsigned)((pairs + 3) / 4), 128, 0, stream>>>(
         a.part_o, a.part_ml, a.out, a.lse, (int)pairs, splits);
     return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Split-KV partials in a buffer the library owns, for callers that cannot
+// allocate device memory themselves (see inkling_attn_decode_static).  The
+// array is part of this module: every device that loads the library holds
+// kDecodeStaticScratchBytes of it until the process exits.  Host code never
+// dereferences the symbol; it asks the runtime for the device address once
+// per device (with that device current) and hands that address to the kernels.
+constexpr size_t kDecodeStaticScratchBytes = (size_t)8 << 20;
+static __device__ __align__(256) unsigned char g_decode_scratch[kDecodeStaticScratchBytes];
+
+cudaError_t decode_static_scratch(void **ptr, size_t *bytes) {
+    static std::mutex mu;
+    static void *addr[64] = {nullptr};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_decode_scratch);
+        if (e != cudaSuccess) return e;
+        addr[dev] = p;
+    }
+    *ptr = addr[dev];
+    *bytes = kDecodeStaticScratchBytes;
+    return cudaSuccess;
 }
 
 }  // namespace inkling
