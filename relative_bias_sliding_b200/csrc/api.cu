@@ -12,6 +12,8 @@ namespace inkling {
 cudaError_t launch_sconv_kv(const inkling_sconv_params &p, cudaStream_t stream);
 cudaError_t launch_attn_prefill(const inkling_prefill_params &p, const CUtensorMap *maps,
                                 cudaStream_t stream);
+cudaError_t launch_attn_prefill_pair(const inkling_prefill_params &p, const CUtensorMap *maps,
+                                     cudaStream_t stream);
 cudaError_t launch_attn_decode(const inkling_decode_params &p, int splits, void *workspace,
                                const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                                cudaStream_t stream);
@@ -196,6 +198,9 @@ inkling_status inkling_attn_prefill(const inkling_prefill_params *p, inkling_str
 
     const cuuint64_t T = (cuuint64_t)p->seq_len, B = (cuuint64_t)p->batch;
     const cuuint64_t Hq = (cuuint64_t)p->num_q_heads, Hkv = (cuuint64_t)p->num_kv_heads;
+    // GQA groups of even size run on CTA pairs (2-SM MMAs sharing every
+    // key/value tile); odd groups on single CTAs
+    const bool pair = ((p->num_q_heads / p->num_kv_heads) % 2) == 0;
     CUtensorMap maps[5];
     {
         // q [B, T, Hq, 128] seen as (d, T, Hq, B)
@@ -206,14 +211,19 @@ inkling_status inkling_attn_prefill(const inkling_prefill_params *p, inkling_str
     }
     const void *kv[2] = {p->k_raw, p->v_raw};
     for (int w = 0; w < 2; ++w) {
-        // raw keys / values [B, T, Hkv, 128] seen as (d, T, Hkv, B): a 128-row
-        // tile box and an 8-row history box
+        // raw keys / values [B, T, Hkv, 128] seen as (d, T, Hkv, B): a tile box
+        // (128 rows, or 64 key rows for a CTA pair) and an 8-row history box
         cuuint64_t dims[4] = {128, T, Hkv, B};
         cuuint64_t str[3] = {Hkv * 256, 256, T * Hkv * 256};
-        cuuint32_t box_t[4] = {64, 128, 1, 1};
+        cuuint32_t box_t[4] = {64, (cuuint32_t)((pair && w == 0) ? 64 : 128), 1, 1};
         cuuint32_t box_h[4] = {64, 8, 1, 1};
         if ((st = make_map(&maps[1 + 2 * w], kv[w], 4, dims, str, box_t)) != INKLING_OK) return st;
         if ((st = make_map(&maps[2 + 2 * w], kv[w], 4, dims, str, box_h)) != INKLING_OK) return st;
+    }
+    if (pair) {
+        cudaError_t e = launch_attn_prefill_pair(*p, maps, (cudaStream_t)stream);
+        if (e != cudaSuccess) return cuda_fail(e, "attn_prefill (CTA pairs) launch");
+        return INKLING_OK;
     }
     cudaError_t e = launch_attn_prefill(*p, maps, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "attn_prefill launch");

@@ -25,20 +25,17 @@
 // The online softmax keeps a reference maximum per row and rescales O only
 // when a row maximum grows by more than 8 (log2 units), which is exact up to
 // rounding because numerator and denominator share the same reference.
-#include "common.cuh"
+#include "prefill_common.cuh"
 
 namespace inkling {
 
-constexpr int kQRows = 256;
 constexpr uint32_t SM_Q = 0;            // 2 tiles x 32 KB
 constexpr uint32_t SM_K = 65536;        // 2 stages x 32 KB
 constexpr uint32_t SM_V = 131072;       // 2 stages x 32 KB
 constexpr uint32_t SM_KH = 196608;      // 2 stages x 2 KB (8 history rows x 2 halves)
 constexpr uint32_t SM_VH = 200704;      // 2 stages x 2 KB
 constexpr uint32_t SM_BIAS = 204800;    // 2 softmax groups x 2 buffers x 4 copies x 264 fp32
-constexpr int kBiasCopy = 264;          // floats per shifted copy (== 8 mod 32: conflict-free)
-constexpr int kBiasBuf = 4 * kBiasCopy;
-constexpr uint32_t SM_BAR = SM_BIAS + 2 * 2 * kBiasBuf * 4;  // mbarriers, tmem base, flags
+constexpr uint32_t SM_BAR = SM_BIAS + kBiasBytes;  // mbarriers, tmem base, flags
 constexpr int kPrefillSmem = SM_BAR + 512 + 1024;
 
 enum {
@@ -55,74 +52,6 @@ enum {
     B_DRAIN = 19,
     B_COUNT = 20
 };
-
-struct PrefillArgs {
-    const float *w_k, *w_v, *bias;
-    uint16_t *out;
-    float *lse;
-    int32_t *status;
-    int B, T, Hq, Hkv, window, d_max, nqb;
-};
-
-// Register split per warpgroup: 2 x 128 softmax threads at 176, 128 sconv
-// threads at 112, 128 producer/MMA/idle threads at 48: 45056 + 14336 + 6144 =
-// 65536 = 512 threads x the 128 registers the kernel launches with (ptxas
-// reports 128), so the increase never waits on registers that do not exist.
-INK_DEV void setmaxnreg_inc176() { asm volatile("setmaxnreg.inc.sync.aligned.u32 176;"); }
-INK_DEV void setmaxnreg_dec112() { asm volatile("setmaxnreg.dec.sync.aligned.u32 112;"); }
-INK_DEV void setmaxnreg_dec48() { asm volatile("setmaxnreg.dec.sync.aligned.u32 48;"); }
-
-// Convert one raw 128-row key or value tile (TMA layout: two 64-column halves
-// of 128 rows x 128 bytes, 128-byte swizzle) into its sconv output, in place,
-// with 64 threads.  Thread v owns 16-byte column c = v % 16 (8 channels) and
-// rows 32g..32g+31, g = v / 16; the 3 rows before its first row come from the
-// tile itself, or for g = 0 from the 8-row history box loaded with the tile.
-// w[tap][pair] holds the taps of channel pairs (2p, 2p+1) of this column.
-INK_DEV void sconv_tile_group(uint32_t tile, uint32_t hist, const f32x2 (&w)[4][4], int v,
-                              int bar_id) {
-    const int c = v & 15, g = v >> 4;
-    const int half = c >> 3, cc = c & 7;
-    const uint32_t tb = tile + half * 16384;
-    f32x2 h3[4], h2[4], h1[4];
-    auto load = [&](uint32_t base, int r, f32x2(&dst)[4]) {
-        const uint4 q = lds128(base + r * 128 + ((cc ^ (r & 7)) << 4));
-        dst[0] = bf2_to_f2(q.x);
-        dst[1] = bf2_to_f2(q.y);
-        dst[2] = bf2_to_f2(q.z);
-        dst[3] = bf2_to_f2(q.w);
-    };
-    if (g == 0) {
-        const uint32_t hb = hist + half * 1024;
-        load(hb, 5, h3);
-        load(hb, 6, h2);
-        load(hb, 7, h1);
-    } else {
-        load(tb, 32 * g - 3, h3);
-        load(tb, 32 * g - 2, h2);
-        load(tb, 32 * g - 1, h1);
-    }
-    named_bar_sync(bar_id, 64);  // every history row read before any row is overwritten
-#pragma unroll 4
-    for (int i = 0; i < 32; ++i) {
-        const int r = 32 * g + i;
-        const uint32_t addr = tb + r * 128 + ((cc ^ (r & 7)) << 4);
-        f32x2 x[4];
-        load(tb, r, x);
-        uint32_t o[4];
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            // same order as the decode append: w3*x[t-3], +w2*x[t-2], +w1*x[t-1], +w0*x[t]
-            f32x2 acc = fmul2(w[3][p], h3[p]);
-            acc = ffma2(w[2][p], h2[p], acc);
-            acc = ffma2(w[1][p], h1[p], acc);
-            acc = ffma2(w[0][p], x[p], acc);
-            o[p] = f2_to_bf2(acc);
-        }
-        sts128(addr, make_uint4(o[0], o[1], o[2], o[3]));
-#pragma unroll
-        for (int p = 0; p < 4; ++p) { h3[p] = h2[p]; h2[p] = h1[p]; h1[p] = x[p]; }
-    }
-}
 
 __global__ void __launch_bounds__(512, 1)
 attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -183,187 +112,19 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
         // ================================================== softmax (2 WGs) ==
         setmaxnreg_inc176();
         const int t = warp >> 2;
-        const int u = threadIdx.x & 127;
-        if (ok[t]) {
-            const uint32_t tl = tbase + ((uint32_t)((warp & 3) * 32) << 16);
-            const uint32_t s_col = tl + t * 128, o_col = tl + 256 + t * 128;
-            const int i = r0[t] + u;
-            const float scale = 0.08838834764831845f;  // 1/sqrt(128)
-            const float kLog2e = 1.4426950408889634f;
-            const float kTau = 5.545177444479562f;       // 8 ln 2
-            const float *bias_h = a.bias + (long)h * (a.d_max + 1);
-            const int W = a.window, Dm = a.d_max, T = a.T;
-            float m_ref = -INFINITY, l = 0.f;
-            float *bias_sm = (float *)(smem + SM_BIAS) + t * 2 * kBiasBuf;
-            const int o_rd = 127 - u, sh = o_rd & 3;  // this row's start in the staged diagonal
-            bool dead = false;
-            int k = 0;
-            for (int n = lo[t]; n <= hi[t]; ++n, ++k) {
-                const int j0 = n * 128;
-                // Stage the bias diagonal of this (query tile, key tile) pair:
-                // R[q] = bias[h, clamp(top - q, 0, d_max)], q = 0..254, top = r0 - j0 + 127,
-                // as 4 copies shifted by 0..3 floats so that row u reads R[127-u+c],
-                // c = 0..127, with aligned 16-byte loads.  Double-buffered by tile parity.
-                float *bb = bias_sm + (k & 1) * kBiasBuf;
-                {
-                    const int top = r0[t] - j0 + 127;
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int q = 2 * u + e;
-                        if (q < 255) {
-                            const float bv = __ldg(bias_h + min(max(top - q, 0), Dm));
-#pragma unroll
-                            for (int s4 = 0; s4 < 4; ++s4)
-                                if (q >= s4) bb[s4 * kBiasCopy + q - s4] = bv;
-                        }
-                    }
-                }
-                named_bar_sync(3 + t, 128);
-                if (!dead) dead = !mbar_wait_warp(&bar[B_SFULL + t], k & 1, abort_flag, a.status);
-                if (dead) continue;  // keep stepping through the group barrier
-                tc_fence_after();
-                uint32_t sr[128];
-                tmem_ld32(s_col + 0, sr + 0);
-                tmem_ld32(s_col + 32, sr + 32);
-                tmem_ld32(s_col + 64, sr + 64);
-                tmem_ld32(s_col + 96, sr + 96);
-                tmem_wait_ld();
-                const float4 *rp = (const float4 *)(bb + sh * kBiasCopy + (o_rd - sh));
-                float x[128];
-                const int dist0 = i - j0;  // distance of key j0 + c is dist0 - c
-                const bool full = (dist0 - 127 >= 0) && (W <= 0 || dist0 < W) && (j0 + 127 < T);
-                if (full) {
-                    const f32x2 sc2 = pk2(scale, scale);
-#pragma unroll
-                    for (int c4 = 0; c4 < 32; ++c4) {
-                        const float4 b4 = rp[c4];
-                        const f32x2 xa = ffma2(pk2(__uint_as_float(sr[4 * c4]),
-                                                   __uint_as_float(sr[4 * c4 + 1])),
-                                               sc2, pk2(b4.x, b4.y));
-                        const f32x2 xb = ffma2(pk2(__uint_as_float(sr[4 * c4 + 2]),
-                                                   __uint_as_float(sr[4 * c4 + 3])),
-                                               sc2, pk2(b4.z, b4.w));
-                        upk2(xa, x[4 * c4], x[4 * c4 + 1]);
-                        upk2(xb, x[4 * c4 + 2], x[4 * c4 + 3]);
-                    }
-                } else {
-#pragma unroll
-                    for (int c4 = 0; c4 < 32; ++c4) {
-                        const float4 b4 = rp[c4];
-                        const float bq[4] = {b4.x, b4.y, b4.z, b4.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int c = 4 * c4 + e;
-                            const int dist = dist0 - c;
-                            const bool allowed = dist >= 0 && (W <= 0 || dist < W) && (j0 + c < T);
-                            x[c] = allowed ? fmaf(__uint_as_float(sr[c]), scale, bq[e]) : -INFINITY;
-                        }
-                    }
-                }
-                // row max: 8 independent chains of 3-input max
-                float m8[8];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) m8[q] = fmaxf(x[2 * q], x[2 * q + 1]);
-#pragma unroll
-                for (int c = 16; c < 128; c += 16)
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) m8[q] = max3f(m8[q], x[c + 2 * q], x[c + 2 * q + 1]);
-                const float mx = fmaxf(max3f(m8[0], m8[1], m8[2]),
-                                       max3f(max3f(m8[3], m8[4], m8[5]), m8[6], m8[7]));
-                // lazy rescale: move the reference only when the max grows by > tau
-                const bool grow = mx > m_ref + kTau;
-                float alpha = 1.f;
-                if (grow) {
-                    alpha = ex2((m_ref - mx) * kLog2e);
-                    l *= alpha;
-                    m_ref = mx;
-                }
-                const float mneg = (m_ref == -INFINITY) ? 0.f : -m_ref * kLog2e;
-                {
-                    const f32x2 l2e2 = pk2(kLog2e, kLog2e), mneg2 = pk2(mneg, mneg);
-                    f32x2 acc[4] = {0ull, 0ull, 0ull, 0ull};
-                    uint32_t pk[64];
-#pragma unroll
-                    for (int c = 0; c < 64; ++c) {
-                        const f32x2 tt = ffma2(pk2(x[2 * c], x[2 * c + 1]), l2e2, mneg2);
-                        float t0, t1;
-                        upk2(tt, t0, t1);
-                        const float p0 = ex2(t0), p1 = ex2(t1);
-                        acc[c & 3] = fadd2(acc[c & 3], pk2(p0, p1));
-                        pk[c] = pack_bf16(p0, p1);
-                    }
-                    tmem_st32(s_col + 0, pk + 0);
-                    tmem_st32(s_col + 32, pk + 32);
-                    const f32x2 s01 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
-                    float la, lb;
-                    upk2(s01, la, lb);
-                    l += la + lb;
-                }
-                // O rescale after P is out of registers (keeps the peak low); the
-                // P.V MMA of this tile is issued only after p_full
-                if (k > 0 && __any_sync(0xffffffffu, grow)) {
-#pragma unroll 1
-                    for (int cb = 0; cb < 4; ++cb) {
-                        uint32_t orr[32];
-                        tmem_ld32(o_col + cb * 32, orr);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
-                        tmem_st32(o_col + cb * 32, orr);
-                    }
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(&bar[B_PFULL + t]);
-            }
-            const bool aborted = dead;
-            // epilogue: O / l -> bf16
-            if (!aborted && mbar_wait_warp(&bar[B_ODONE + t], 0, abort_flag, a.status)) {
-                tc_fence_after();
-                const float inv = (l > 0.f) ? 1.f / l : 0.f;
-                uint4 *dst = (uint4 *)(a.out + (((long)b * T + i) * a.Hq + h) * 128);
-#pragma unroll
-                for (int cb = 0; cb < 4; ++cb) {
-                    uint32_t orr[32];
-                    tmem_ld32(o_col + cb * 32, orr);
-                    tmem_wait_ld();
-                    if (i < T) {
-#pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            uint4 v;
-                            v.x = pack_bf16(__uint_as_float(orr[q4 * 8 + 0]) * inv,
-                                            __uint_as_float(orr[q4 * 8 + 1]) * inv);
-                            v.y = pack_bf16(__uint_as_float(orr[q4 * 8 + 2]) * inv,
-                                            __uint_as_float(orr[q4 * 8 + 3]) * inv);
-                            v.z = pack_bf16(__uint_as_float(orr[q4 * 8 + 4]) * inv,
-                                            __uint_as_float(orr[q4 * 8 + 5]) * inv);
-                            v.w = pack_bf16(__uint_as_float(orr[q4 * 8 + 6]) * inv,
-                                            __uint_as_float(orr[q4 * 8 + 7]) * inv);
-                            dst[cb * 4 + q4] = v;
-                        }
-                    }
-                }
-                if (a.lse && i < T)
-                    a.lse[((long)b * a.Hq + h) * T + i] = (l > 0.f) ? m_ref + __logf(l) : -INFINITY;
-            }
-        }
+        if (ok[t])
+            softmax_role(a, (float *)(smem + SM_BIAS) + t * 2 * kBiasBuf, &bar[B_SFULL],
+                         &bar[B_ODONE], abort_flag, tbase, t, b, h, r0[t], lo[t], hi[t], 3 + t,
+                         [&](int tt) { mbar_arrive(&bar[B_PFULL + tt]); });
     } else if (warp < 12) {
-        // ============================================ sconv transform (WG2) ==
+        // ========================== sconv transform: warps 8-9 keys, 10-11 values ==
         setmaxnreg_dec112();
         const bool is_v = warp >= 10;
         const int v = threadIdx.x - (is_v ? 320 : 256);
         const int bar_id = is_v ? 2 : 1;
-        // taps of this thread's 8 channels, as channel pairs, held for the whole block
+        // taps of this thread's 8 channels, held for the whole block
         f32x2 w[4][4];
-        {
-            const float *wg = (is_v ? a.w_v : a.w_k) + ((long)kvh * 128 + 8 * (v & 15)) * 4;
-#pragma unroll
-            for (int p = 0; p < 4; ++p)
-#pragma unroll
-                for (int tap = 0; tap < 4; ++tap)
-                    w[tap][p] = pk2(__ldg(wg + (2 * p) * 4 + tap), __ldg(wg + (2 * p + 1) * 4 + tap));
-        }
+        load_taps(w, (is_v ? a.w_v : a.w_k) + ((long)kvh * 128 + 8 * (v & 15)) * 4);
         uint64_t *raw_full = &bar[is_v ? B_VRAW : B_KRAW];
         uint64_t *ready = &bar[is_v ? B_VREADY : B_KREADY];
         const uint32_t tiles = sb + (is_v ? SM_V : SM_K);
@@ -377,7 +138,9 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                 named_bar_sync(bar_id, 64);  // keep the group's barrier count matched
                 continue;
             }
-            sconv_tile_group(tiles + st * 32768, hists + st * 2048, w, v, bar_id);
+            // thread v: column v % 16, rows 32 (v / 16) .. +32 of the 128-row tile
+            sconv_rows(tiles + st * 32768, hists + st * 2048, 16384, w, v & 15, 32 * (v >> 4), 32,
+                       bar_id, 64);
             fence_proxy_async_smem();
             mbar_arrive(&ready[st]);
         }

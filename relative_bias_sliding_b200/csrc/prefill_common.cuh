@@ -1,0 +1,267 @@
+// prefill_common.cuh — pieces shared by the two prefill kernels (one CTA per
+// query block, or a 2-CTA cluster sharing every key/value tile): arguments,
+// the register split, the in-place sconv transform of a raw key/value tile and
+// the softmax role of one 128-row query tile.
+#pragma once
+
+#include "common.cuh"
+
+namespace inkling {
+
+constexpr int kQRows = 256;     // query rows per CTA: two 128-row tiles
+constexpr int kBiasCopy = 264;  // floats per shifted bias copy (== 8 mod 32: conflict-free)
+constexpr int kBiasBuf = 4 * kBiasCopy;
+constexpr int kBiasBytes = 2 * 2 * kBiasBuf * 4;  // 2 query tiles x 2 buffers
+
+struct PrefillArgs {
+    const float *w_k, *w_v, *bias;
+    uint16_t *out;
+    float *lse;
+    int32_t *status;
+    int B, T, Hq, Hkv, window, d_max, nqb;
+};
+
+// Register split per warpgroup: 2 x 128 softmax threads at 176, 128 sconv
+// threads at 112, 128 producer/MMA/idle threads at 48: 45056 + 14336 + 6144 =
+// 65536 = 512 threads x the 128 registers the kernels launch with (ptxas
+// reports 128), so the increase never waits on registers that do not exist.
+INK_DEV void setmaxnreg_inc176() { asm volatile("setmaxnreg.inc.sync.aligned.u32 176;"); }
+INK_DEV void setmaxnreg_dec112() { asm volatile("setmaxnreg.dec.sync.aligned.u32 112;"); }
+INK_DEV void setmaxnreg_dec48() { asm volatile("setmaxnreg.dec.sync.aligned.u32 48;"); }
+
+// Taps of 8 consecutive channels starting at `wg` ([C, 4] fp32), as channel
+// pairs: w[tap][p] = (w[2p][tap], w[2p+1][tap]).
+INK_DEV void load_taps(f32x2 (&w)[4][4], const float *wg) {
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+#pragma unroll
+        for (int tap = 0; tap < 4; ++tap)
+            w[tap][p] = pk2(__ldg(wg + (2 * p) * 4 + tap), __ldg(wg + (2 * p + 1) * 4 + tap));
+}
+
+// In-place sconv of rows [row0, row0 + nrows) of one 16-byte column of a raw
+// key/value tile.  The tile is TMA-loaded with 128-byte swizzle as 64-column
+// halves of 128-byte rows (`half_bytes` apart); the 8-row history box (rows
+// -8..-1, halves 1 KB apart) supplies the 3 rows before row 0.  Column `c`
+// (0..15) selects half c/8 and chunk c%8.  All `nthreads` threads of the group
+// read their 3 history rows before a named barrier; only then is anything
+// overwritten.
+INK_DEV void sconv_rows(uint32_t tile, uint32_t hist, uint32_t half_bytes, const f32x2 (&w)[4][4],
+                        int c, int row0, int nrows, int bar_id, int nthreads) {
+    const int half = c >> 3, cc = c & 7;
+    const uint32_t tb = tile + half * half_bytes;
+    f32x2 h3[4], h2[4], h1[4];
+    auto load = [&](uint32_t base, int r, f32x2(&dst)[4]) {
+        const uint4 q = lds128(base + r * 128 + ((cc ^ (r & 7)) << 4));
+        dst[0] = bf2_to_f2(q.x);
+        dst[1] = bf2_to_f2(q.y);
+        dst[2] = bf2_to_f2(q.z);
+        dst[3] = bf2_to_f2(q.w);
+    };
+    if (row0 == 0) {
+        const uint32_t hb = hist + half * 1024;
+        load(hb, 5, h3);
+        load(hb, 6, h2);
+        load(hb, 7, h1);
+    } else {
+        load(tb, row0 - 3, h3);
+        load(tb, row0 - 2, h2);
+        load(tb, row0 - 1, h1);
+    }
+    named_bar_sync(bar_id, nthreads);  // every history row read before any row is overwritten
+#pragma unroll 4
+    for (int i = 0; i < nrows; ++i) {
+        const int r = row0 + i;
+        const uint32_t addr = tb + r * 128 + ((cc ^ (r & 7)) << 4);
+        f32x2 x[4];
+        load(tb, r, x);
+        uint32_t o[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            // same order as the decode append: w3*x[t-3], +w2*x[t-2], +w1*x[t-1], +w0*x[t]
+            f32x2 acc = fmul2(w[3][p], h3[p]);
+            acc = ffma2(w[2][p], h2[p], acc);
+            acc = ffma2(w[1][p], h1[p], acc);
+            acc = ffma2(w[0][p], x[p], acc);
+            o[p] = f2_to_bf2(acc);
+        }
+        sts128(addr, make_uint4(o[0], o[1], o[2], o[3]));
+#pragma unroll
+        for (int p = 0; p < 4; ++p) { h3[p] = h2[p]; h2[p] = h1[p]; h1[p] = x[p]; }
+    }
+}
+
+// Softmax of one 128-row query tile (the calling warpgroup; thread = row =
+// TMEM lane), over key tiles lo..hi, then the epilogue.  S lives in TMEM
+// columns [128t, 128t+128), O in [256+128t, ...); P (bf16) is written over the
+// first 64 columns of S.  `signal_p(t)` is called by every thread once its P
+// and O updates are complete and fenced; it must tell the MMA issuer.
+// `bias_sm` holds this tile's two bias-diagonal buffers; `bar_id` is a named
+// barrier private to this warpgroup.
+template <class SignalP>
+INK_DEV void softmax_role(const PrefillArgs &a, float *bias_sm, uint64_t *s_full, uint64_t *o_done,
+                          volatile int *abort_flag, uint32_t tbase, int t, int b, int h, int r0,
+                          int lo, int hi, int bar_id, SignalP signal_p) {
+    const int u = threadIdx.x & 127;
+    const uint32_t tl = tbase + ((uint32_t)(((threadIdx.x >> 5) & 3) * 32) << 16);
+    const uint32_t s_col = tl + t * 128, o_col = tl + 256 + t * 128;
+    const int i = r0 + u;
+    const float scale = 0.08838834764831845f;  // 1/sqrt(128)
+    const float kLog2e = 1.4426950408889634f;
+    const float kTau = 5.545177444479562f;     // 8 ln 2
+    const float *bias_h = a.bias + (long)h * (a.d_max + 1);
+    const int W = a.window, Dm = a.d_max, T = a.T;
+    float m_ref = -INFINITY, l = 0.f;
+    const int o_rd = 127 - u, sh = o_rd & 3;  // this row's start in the staged diagonal
+    bool dead = false;
+    int k = 0;
+    for (int n = lo; n <= hi; ++n, ++k) {
+        const int j0 = n * 128;
+        // Stage the bias diagonal of this (query tile, key tile) pair:
+        // R[q] = bias[h, clamp(top - q, 0, d_max)], q = 0..254, top = r0 - j0 + 127,
+        // as 4 copies shifted by 0..3 floats so that row u reads R[127-u+c],
+        // c = 0..127, with aligned 16-byte loads.  Double-buffered by tile parity.
+        float *bb = bias_sm + (k & 1) * kBiasBuf;
+        {
+            const int top = r0 - j0 + 127;
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int q = 2 * u + e;
+                if (q < 255) {
+                    const float bv = __ldg(bias_h + min(max(top - q, 0), Dm));
+#pragma unroll
+                    for (int s4 = 0; s4 < 4; ++s4)
+                        if (q >= s4) bb[s4 * kBiasCopy + q - s4] = bv;
+                }
+            }
+        }
+        named_bar_sync(bar_id, 128);
+        if (!dead) dead = !mbar_wait_warp(&s_full[t], k & 1, abort_flag, a.status);
+        if (dead) continue;  // keep stepping through the group barrier
+        tc_fence_after();
+        uint32_t sr[128];
+        tmem_ld32(s_col + 0, sr + 0);
+        tmem_ld32(s_col + 32, sr + 32);
+        tmem_ld32(s_col + 64, sr + 64);
+        tmem_ld32(s_col + 96, sr + 96);
+        tmem_wait_ld();
+        const float4 *rp = (const float4 *)(bb + sh * kBiasCopy + (o_rd - sh));
+        float x[128];
+        const int dist0 = i - j0;  // distance of key j0 + c is dist0 - c
+        const bool full = (dist0 - 127 >= 0) && (W <= 0 || dist0 < W) && (j0 + 127 < T);
+        // logits and row max, 32 columns at a time: the 8 bias loads of a batch
+        // are issued together, and 8 independent 3-input max chains run
+        // alongside
+        float m8[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
+#pragma unroll
+        for (int cb = 0; cb < 4; ++cb) {
+            float4 b4[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) b4[j] = rp[cb * 8 + j];
+            if (full) {
+                const f32x2 sc2 = pk2(scale, scale);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int c = 32 * cb + 4 * j;
+                    const f32x2 xa = ffma2(pk2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])),
+                                           sc2, pk2(b4[j].x, b4[j].y));
+                    const f32x2 xb = ffma2(pk2(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3])),
+                                           sc2, pk2(b4[j].z, b4[j].w));
+                    upk2(xa, x[c], x[c + 1]);
+                    upk2(xb, x[c + 2], x[c + 3]);
+                    m8[j] = max3f(max3f(m8[j], x[c], x[c + 1]), x[c + 2], x[c + 3]);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float bq[4] = {b4[j].x, b4[j].y, b4[j].z, b4[j].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int c = 32 * cb + 4 * j + e;
+                        const int dist = dist0 - c;
+                        const bool allowed = dist >= 0 && (W <= 0 || dist < W) && (j0 + c < T);
+                        x[c] = allowed ? fmaf(__uint_as_float(sr[c]), scale, bq[e]) : -INFINITY;
+                    }
+                    const int c = 32 * cb + 4 * j;
+                    m8[j] = max3f(max3f(m8[j], x[c], x[c + 1]), x[c + 2], x[c + 3]);
+                }
+            }
+        }
+        const float mx =
+            fmaxf(max3f(m8[0], m8[1], m8[2]), max3f(max3f(m8[3], m8[4], m8[5]), m8[6], m8[7]));
+        // lazy rescale: move the reference only when the max grows by > tau
+        const bool grow = mx > m_ref + kTau;
+        float alpha = 1.f;
+        if (grow) {
+            alpha = ex2((m_ref - mx) * kLog2e);
+            l *= alpha;
+            m_ref = mx;
+        }
+        const float mneg = (m_ref == -INFINITY) ? 0.f : -m_ref * kLog2e;
+        {
+            const f32x2 l2e2 = pk2(kLog2e, kLog2e), mneg2 = pk2(mneg, mneg);
+            f32x2 acc[4] = {0ull, 0ull, 0ull, 0ull};
+            uint32_t pk[64];
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+                const f32x2 tt = ffma2(pk2(x[2 * c], x[2 * c + 1]), l2e2, mneg2);
+                float t0, t1;
+                upk2(tt, t0, t1);
+                const float p0 = ex2(t0), p1 = ex2(t1);
+                acc[c & 3] = fadd2(acc[c & 3], pk2(p0, p1));
+                pk[c] = pack_bf16(p0, p1);
+            }
+            tmem_st32(s_col + 0, pk + 0);
+            tmem_st32(s_col + 32, pk + 32);
+            const f32x2 s01 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+            float la, lb;
+            upk2(s01, la, lb);
+            l += la + lb;
+        }
+        // O rescale after P is out of registers (keeps the peak low); the P.V
+        // MMA of this tile is issued only after the P signal
+        if (k > 0 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll 1
+            for (int cb = 0; cb < 4; ++cb) {
+                uint32_t orr[32];
+                tmem_ld32(o_col + cb * 32, orr);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
+                tmem_st32(o_col + cb * 32, orr);
+            }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        signal_p(t);
+    }
+    // epilogue: O / l -> bf16
+    if (!dead && mbar_wait_warp(&o_done[t], 0, abort_flag, a.status)) {
+        tc_fence_after();
+        const float inv = (l > 0.f) ? 1.f / l : 0.f;
+        uint4 *dst = (uint4 *)(a.out + (((long)b * T + i) * a.Hq + h) * 128);
+#pragma unroll
+        for (int cb = 0; cb < 4; ++cb) {
+            uint32_t orr[32];
+            tmem_ld32(o_col + cb * 32, orr);
+            tmem_wait_ld();
+            if (i < T) {
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    uint4 v;
+                    v.x = pack_bf16(__uint_as_float(orr[q4 * 8 + 0]) * inv, __uint_as_float(orr[q4 * 8 + 1]) * inv);
+                    v.y = pack_bf16(__uint_as_float(orr[q4 * 8 + 2]) * inv, __uint_as_float(orr[q4 * 8 + 3]) * inv);
+                    v.z = pack_bf16(__uint_as_float(orr[q4 * 8 + 4]) * inv, __uint_as_float(orr[q4 * 8 + 5]) * inv);
+                    v.w = pack_bf16(__uint_as_float(orr[q4 * 8 + 6]) * inv, __uint_as_float(orr[q4 * 8 + 7]) * inv);
+                    dst[cb * 4 + q4] = v;
+                }
+            }
+        }
+        if (a.lse && i < T)
+            a.lse[((long)b * a.Hq + h) * T + i] = (l > 0.f) ? m_ref + __logf(l) : -INFINITY;
+    }
+}
+
+}  // namespace inkling
