@@ -36,6 +36,15 @@ DEFAULT_PREFILL = "prefill_swa_b4_t8192"
 DEFAULT_DECODE = "decode_swa_s64"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one
+# ncu capture of the current kernels on a smaller cut of the same workload,
+# scaled by the units processed (profiles/ holds the summaries and commands).
+# Set an entry to None when its kernel changes until it is captured again.
+MEASURED_TRAFFIC = {
+    "prefill_swa_b4_t8192": 4 * 269.2e6,   # B1 capture x 4 batches
+    "decode_swa_s64": 1.049 * 1061945344,  # 16-sequence capture: traffic / KV bytes = 1.049
+}
+
 
 # ------------------------------------------------------------ distributed --
 
@@ -91,7 +100,7 @@ class ClockSampler:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.fh,
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.fh,
                 stderr=subprocess.DEVNULL)
             time.sleep(0.3)
         except Exception:
@@ -353,7 +362,7 @@ def oracle_decode_sample(spec, seconds, seed=0):
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=150)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=None,
@@ -471,9 +480,10 @@ def main():
         tflops = pre.flops / (pre_ms * 1e-3) / 1e12 * world
         peak = peaks["bf16_tflops_sustained"]
         line.update({"value": tflops, "unit": "TFLOP/s"})
-        line["roofline"] = {"bound": "tensor", "kernel": "attn_prefill_kernel",
+        line["roofline"] = {"bound": "tensor", "kernel": "attn_prefill_pair_kernel",
                             "achieved": tflops / world, "peak": peak, "unit": "TFLOP/s",
-                            "frac": tflops / world / peak, "traffic": None,
+                            "frac": tflops / world / peak,
+                            "traffic": MEASURED_TRAFFIC.get(pre.spec.name),
                             "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed "
                                            f"inside a long step loop)"}
     if dec:
@@ -487,7 +497,8 @@ def main():
                    "roofline": {"bound": "hbm", "kernel": "decode_split_kernel + combine",
                                 "achieved": kern_gbs, "peak": peaks["hbm_gbs"],
                                 "unit": "GB/s", "frac": kern_gbs / peaks["hbm_gbs"],
-                                "traffic": None, "peak_source": f"{peak_src} hbm_gbs"}}
+                                "traffic": MEASURED_TRAFFIC.get(dec.spec.name),
+                                "peak_source": f"{peak_src} hbm_gbs"}}
         if pre:
             line["decode"] = dec_obj
         else:
