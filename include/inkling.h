@@ -70,6 +70,16 @@ const char *inkling_last_error(void);
 /* Library version, major*10000 + minor*100 + patch. */
 int inkling_version(void);
 
+/* Self-test of failure detection (the pages have no counterpart).  Every wait
+ * inside the kernels is bounded: when a wait runs out, the kernel ORs
+ * INKLING_STATUS_TIMEOUT into the status word and returns instead of hanging,
+ * and the CUDA context stays usable.  This call launches one block that waits,
+ * with a limit of limit_us microseconds (1 .. 10^7), on a barrier that nothing
+ * will ever arrive on, so the caller can check that path end to end.  status:
+ * device int32, zeroed by the caller. */
+inkling_status inkling_selftest_wait_timeout(int32_t *status, uint32_t limit_us,
+                                             inkling_stream_t stream);
+
 /* --------------------------------------------------------------------------
  * inkling_sconv_kv — decode-side sconv append (Overview, "Short convolution":
  * the sconv on keys and values, with its state kept as a sliding-window

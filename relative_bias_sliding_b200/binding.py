@@ -25,6 +25,7 @@ BLOCK_SIZE = 128
 EXPORTED = (
     "inkling_last_error",
     "inkling_version",
+    "inkling_selftest_wait_timeout",
     "inkling_sconv_kv",
     "inkling_attn_prefill",
     "inkling_attn_decode_workspace_bytes",
@@ -80,6 +81,8 @@ def load_library(path: str = LIB_PATH):
         lib = ctypes.CDLL(path)
         lib.inkling_last_error.restype = ctypes.c_char_p
         lib.inkling_version.restype = ctypes.c_int
+        lib.inkling_selftest_wait_timeout.argtypes = [_P, ctypes.c_uint32, _P]
+        lib.inkling_selftest_wait_timeout.restype = ctypes.c_int
         lib.inkling_sconv_kv.argtypes = [ctypes.POINTER(SconvParams), _P]
         lib.inkling_sconv_kv.restype = ctypes.c_int
         lib.inkling_attn_prefill.argtypes = [ctypes.POINTER(PrefillParams), _P]
@@ -263,3 +266,9 @@ def attn_decode_static(q, k_cache, v_cache, block_table, seq_lens, bias, window=
                        num_splits)
     _check(load_library().inkling_attn_decode_static(ctypes.byref(p), _stream(stream)))
     return out
+
+
+def selftest_wait_timeout(status, limit_us=50000, stream=None):
+    """Launch a block whose bounded wait must run out (see inkling.h)."""
+    _dev(status, torch.int32, "status")
+    _check(load_library().inkling_selftest_wait_timeout(_ptr(status), int(limit_us), _stream(stream)))

@@ -18,6 +18,7 @@ cudaError_t launch_attn_decode(const inkling_decode_params &p, int splits, void 
                                const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                                cudaStream_t stream);
 cudaError_t decode_static_scratch(void **ptr, size_t *bytes);
+cudaError_t launch_wait_timeout_probe(int32_t *status, uint32_t limit_us, cudaStream_t stream);
 }  // namespace inkling
 
 using namespace inkling;
@@ -146,6 +147,19 @@ extern "C" {
 const char *inkling_last_error(void) { return g_err; }
 
 int inkling_version(void) { return 100; }
+
+inkling_status inkling_selftest_wait_timeout(int32_t *status, uint32_t limit_us,
+                                             inkling_stream_t stream) {
+    g_err[0] = 0;
+    if (!status) return fail(INKLING_ERR_INVALID, "status is NULL");
+    if (limit_us == 0 || limit_us > 10000000u)
+        return fail(INKLING_ERR_INVALID, "limit_us must be in [1, 10^7]");
+    inkling_status st = check_device(nullptr);
+    if (st != INKLING_OK) return st;
+    cudaError_t e = launch_wait_timeout_probe(status, limit_us, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "wait timeout probe launch");
+    return INKLING_OK;
+}
 
 inkling_status inkling_sconv_kv(const inkling_sconv_params *p, inkling_stream_t stream) {
     g_err[0] = 0;

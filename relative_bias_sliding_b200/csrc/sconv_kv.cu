@@ -85,4 +85,25 @@ cudaError_t launch_sconv_kv(const inkling_sconv_params &p, cudaStream_t stream) 
     return cudaGetLastError();
 }
 
+// Self-test of the bounded waits every kernel of this library uses: one thread
+// waits on an mbarrier phase that nothing will complete, with a short limit;
+// the wait gives up, reports INKLING_STATUS_TIMEOUT and the kernel returns.
+__global__ void wait_timeout_probe_kernel(int32_t *status, uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, &abort_flag, status, limit_ns);
+    __syncthreads();
+}
+
+cudaError_t launch_wait_timeout_probe(int32_t *status, uint32_t limit_us, cudaStream_t stream) {
+    wait_timeout_probe_kernel<<<1, 32, 0, stream>>>(status, (uint64_t)limit_us * 1000ull);
+    return cudaGetLastError();
+}
+
 }  // namespace inkling
