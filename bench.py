@@ -24,6 +24,7 @@ import json
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -41,7 +42,6 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # scaled by the units processed (profiles/ holds the summaries and commands).
 # Set an entry to None when its kernel changes until it is captured again.
 MEASURED_TRAFFIC = {
-    "prefill_swa_b4_t8192": 4 * 269.2e6,   # B1 capture x 4 batches
     "decode_swa_s64": 1.049 * 1061945344,  # 16-sequence capture: traffic / KV bytes = 1.049
 }
 
@@ -89,10 +89,15 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index):
+    def __init__(self, gpu_index, log_dir=None):
+        # the raw samples go to <log_dir>/clocks_gpu<i>.csv when a directory
+        # is given, else to a temporary file
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+        if log_dir:
+            self.path = os.path.join(log_dir, f"clocks_gpu{gpu_index}.csv")
+        else:
+            self.path = os.path.join(tempfile.gettempdir(), f"inkling_clocks_{os.getpid()}.csv")
 
     def __enter__(self):
         try:
@@ -369,6 +374,8 @@ def parse():
                     help="a single workload name from relative_bias_sliding_b200.inputs.WORKLOADS")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clocks-log-dir", default=None,
+                    help="keep the raw nvidia-smi clock samples in this directory")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
 
@@ -444,7 +451,7 @@ def main():
     stream.synchronize()
     barrier(dist, device)
     torch.cuda.synchronize()
-    with ClockSampler(local) as clocks:
+    with ClockSampler(local, args.clocks_log_dir) as clocks:
         barrier(dist, device)
         torch.cuda.synchronize()
         t_start = torch.cuda.Event(enable_timing=True)

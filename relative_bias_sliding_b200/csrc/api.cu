@@ -215,13 +215,14 @@ inkling_status inkling_attn_prefill(const inkling_prefill_params *p, inkling_str
     // GQA groups of even size run on CTA pairs (2-SM MMAs sharing every
     // key/value tile); odd groups on single CTAs
     const bool pair = ((p->num_q_heads / p->num_kv_heads) % 2) == 0;
-    CUtensorMap maps[5];
+    CUtensorMap maps[6];
     {
-        // q [B, T, Hq, 128] seen as (d, T, Hq, B)
+        // q and out [B, T, Hq, 128] seen as (d, T, Hq, B)
         cuuint64_t dims[4] = {128, T, Hq, B};
         cuuint64_t str[3] = {Hq * 256, 256, T * Hq * 256};
         cuuint32_t box[4] = {64, 128, 1, 1};
         if ((st = make_map(&maps[0], p->q, 4, dims, str, box)) != INKLING_OK) return st;
+        if ((st = make_map(&maps[5], p->out, 4, dims, str, box)) != INKLING_OK) return st;
     }
     const void *kv[2] = {p->k_raw, p->v_raw};
     for (int w = 0; w < 2; ++w) {

@@ -58,7 +58,8 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_kh,
                     const __grid_constant__ CUtensorMap tm_v,
-                    const __grid_constant__ CUtensorMap tm_vh, const PrefillArgs a) {
+                    const __grid_constant__ CUtensorMap tm_vh,
+                    const __grid_constant__ CUtensorMap tm_out, const PrefillArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sb = smem_u32(smem);
@@ -115,6 +116,7 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (ok[t])
             softmax_role(a, (float *)(smem + SM_BIAS) + t * 2 * kBiasBuf, &bar[B_SFULL],
                          &bar[B_ODONE], abort_flag, tbase, t, b, h, r0[t], lo[t], hi[t], 3 + t,
+                         smem + SM_Q + t * 32768, &tm_out,
                          [&](int tt) { mbar_arrive(&bar[B_PFULL + tt]); });
     } else if (warp < 12) {
         // ========================== sconv transform: warps 8-9 keys, 10-11 values ==
@@ -295,7 +297,7 @@ cudaError_t launch_attn_prefill(const inkling_prefill_params &p, const CUtensorM
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kPrefillSmem);
     if (e != cudaSuccess) return e;
     attn_prefill_kernel<<<(unsigned)grid, 512, kPrefillSmem, stream>>>(maps[0], maps[1], maps[2],
-                                                                      maps[3], maps[4], a);
+                                                                      maps[3], maps[4], maps[5], a);
     return cudaGetLastError();
 }
 

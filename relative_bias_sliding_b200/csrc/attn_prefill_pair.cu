@@ -55,7 +55,8 @@ attn_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k64,
                          const __grid_constant__ CUtensorMap tm_kh,
                          const __grid_constant__ CUtensorMap tm_v,
-                         const __grid_constant__ CUtensorMap tm_vh, const PrefillArgs a) {
+                         const __grid_constant__ CUtensorMap tm_vh,
+                    const __grid_constant__ CUtensorMap tm_out, const PrefillArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sb = smem_u32(smem);
@@ -116,7 +117,8 @@ attn_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int t = warp >> 2;
         if (ok[t])
             softmax_role(a, (float *)(smem + PBIAS) + t * 2 * kBiasBuf, &bar[S_FULL], &bar[O_DONE],
-                         abort_flag, tbase, t, b, h, r0[t], lo[t], hi[t], 3 + t, [&](int tt) {
+                         abort_flag, tbase, t, b, h, r0[t], lo[t], hi[t], 3 + t,
+                         smem + PQ + t * 32768, &tm_out, [&](int tt) {
                              __syncwarp();
                              if (lane == 0) mbar_arrive_cta_relaxed(&bar[P_FULL + tt], 0);
                          });
@@ -328,7 +330,7 @@ cudaError_t launch_attn_prefill_pair(const inkling_prefill_params &p, const CUte
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, attn_prefill_pair_kernel, maps[0], maps[1], maps[2], maps[3],
-                           maps[4], a);
+                           maps[4], maps[5], a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -118,6 +118,18 @@ INK_DEV void tma_load_4d(void *dst, const CUtensorMap *m, uint64_t *bar, int x, 
         : "memory");
 }
 
+// bulk tensor store shared -> global (tile mode); elements outside the tensor
+// are not written
+INK_DEV void tma_store_4d(const CUtensorMap *m, const void *src, int x, int y, int z, int w) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(m),
+        "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z), "r"(w)
+        : "memory");
+}
+INK_DEV void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until every committed bulk store of this thread has completed
+INK_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // generic-proxy shared-memory writes -> visible to the async proxy (tensor core)
 INK_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 

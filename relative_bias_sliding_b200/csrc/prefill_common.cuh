@@ -98,10 +98,15 @@ INK_DEV void sconv_rows(uint32_t tile, uint32_t hist, uint32_t half_bytes, const
 // and O updates are complete and fenced; it must tell the MMA issuer.
 // `bias_sm` holds this tile's two bias-diagonal buffers; `bar_id` is a named
 // barrier private to this warpgroup.
+// The epilogue stages the normalised bf16 O tile in `stage` (the query tile's
+// shared-memory buffer, free once the last QK^T of the tile has completed) in
+// the same 128-byte-swizzled layout, and one thread writes it with two bulk
+// tensor stores through `tm_out` (rows past the sequence end are clipped).
 template <class SignalP>
 INK_DEV void softmax_role(const PrefillArgs &a, float *bias_sm, uint64_t *s_full, uint64_t *o_done,
                           volatile int *abort_flag, uint32_t tbase, int t, int b, int h, int r0,
-                          int lo, int hi, int bar_id, SignalP signal_p) {
+                          int lo, int hi, int bar_id, uint8_t *stage, const CUtensorMap *tm_out,
+                          SignalP signal_p) {
     const int u = threadIdx.x & 127;
     const uint32_t tl = tbase + ((uint32_t)(((threadIdx.x >> 5) & 3) * 32) << 16);
     const uint32_t s_col = tl + t * 128, o_col = tl + 256 + t * 128;
@@ -237,30 +242,38 @@ INK_DEV void softmax_role(const PrefillArgs &a, float *bias_sm, uint64_t *s_full
         tc_fence_before();
         signal_p(t);
     }
-    // epilogue: O / l -> bf16
-    if (!dead && mbar_wait_warp(&o_done[t], 0, abort_flag, a.status)) {
+    // epilogue: O / l -> bf16, staged in shared memory, one bulk store per half
+    const bool have_o = !dead && mbar_wait_warp(&o_done[t], 0, abort_flag, a.status);
+    if (have_o) {
         tc_fence_after();
         const float inv = (l > 0.f) ? 1.f / l : 0.f;
-        uint4 *dst = (uint4 *)(a.out + (((long)b * T + i) * a.Hq + h) * 128);
 #pragma unroll
         for (int cb = 0; cb < 4; ++cb) {
             uint32_t orr[32];
             tmem_ld32(o_col + cb * 32, orr);
             tmem_wait_ld();
-            if (i < T) {
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    uint4 v;
-                    v.x = pack_bf16(__uint_as_float(orr[q4 * 8 + 0]) * inv, __uint_as_float(orr[q4 * 8 + 1]) * inv);
-                    v.y = pack_bf16(__uint_as_float(orr[q4 * 8 + 2]) * inv, __uint_as_float(orr[q4 * 8 + 3]) * inv);
-                    v.z = pack_bf16(__uint_as_float(orr[q4 * 8 + 4]) * inv, __uint_as_float(orr[q4 * 8 + 5]) * inv);
-                    v.w = pack_bf16(__uint_as_float(orr[q4 * 8 + 6]) * inv, __uint_as_float(orr[q4 * 8 + 7]) * inv);
-                    dst[cb * 4 + q4] = v;
-                }
+            for (int q4 = 0; q4 < 4; ++q4) {
+                uint4 v;
+                v.x = pack_bf16(__uint_as_float(orr[q4 * 8 + 0]) * inv, __uint_as_float(orr[q4 * 8 + 1]) * inv);
+                v.y = pack_bf16(__uint_as_float(orr[q4 * 8 + 2]) * inv, __uint_as_float(orr[q4 * 8 + 3]) * inv);
+                v.z = pack_bf16(__uint_as_float(orr[q4 * 8 + 4]) * inv, __uint_as_float(orr[q4 * 8 + 5]) * inv);
+                v.w = pack_bf16(__uint_as_float(orr[q4 * 8 + 6]) * inv, __uint_as_float(orr[q4 * 8 + 7]) * inv);
+                const int c = cb * 4 + q4;  // 16-byte chunk of the 256-byte row
+                *(uint4 *)(stage + (c >> 3) * 16384 + u * 128 + (((c & 7) ^ (u & 7)) << 4)) = v;
             }
         }
         if (a.lse && i < T)
             a.lse[((long)b * a.Hq + h) * T + i] = (l > 0.f) ? m_ref + __logf(l) : -INFINITY;
+        fence_proxy_async_smem();
+    }
+    // every warp of the group reaches this barrier (have_o is uniform per warp)
+    named_bar_sync(bar_id, 128);
+    if (u == 0 && have_o && !*abort_flag) {
+        tma_store_4d(tm_out, stage, 0, r0, h, b);
+        tma_store_4d(tm_out, stage + 16384, 64, r0, h, b);
+        bulk_commit_group();
+        bulk_wait_all();
     }
 }
 
