@@ -111,7 +111,7 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
 
     if (warp < 8) {
         // ================================================== softmax (2 WGs) ==
-        setmaxnreg_inc176();
+        setmaxnreg_inc184();
         const int t = warp >> 2;
         if (ok[t])
             softmax_role(a, (float *)(smem + SM_BIAS) + t * 2 * kBiasBuf, &bar[B_SFULL],
@@ -120,7 +120,7 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                          [&](int tt) { mbar_arrive(&bar[B_PFULL + tt]); });
     } else if (warp < 12) {
         // ========================== sconv transform: warps 8-9 keys, 10-11 values ==
-        setmaxnreg_dec112();
+        setmaxnreg_dec80();
         const bool is_v = warp >= 10;
         const int v = threadIdx.x - (is_v ? 320 : 256);
         const int bar_id = is_v ? 2 : 1;
@@ -147,7 +147,7 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
             mbar_arrive(&ready[st]);
         }
     } else {
-        setmaxnreg_dec48();
+        setmaxnreg_dec64();
         if (warp == 12 && lane == 0) {
             // ============================================== TMA producer ==
             tma_prefetch_desc(&tm_q);

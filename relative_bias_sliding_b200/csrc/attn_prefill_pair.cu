@@ -113,7 +113,7 @@ attn_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
 
     if (warp < 8) {
         // ================================================== softmax (2 WGs) ==
-        setmaxnreg_inc176();
+        setmaxnreg_inc184();
         const int t = warp >> 2;
         if (ok[t])
             softmax_role(a, (float *)(smem + PBIAS) + t * 2 * kBiasBuf, &bar[S_FULL], &bar[O_DONE],
@@ -124,7 +124,7 @@ attn_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                          });
     } else if (warp < 12) {
         // ==================== sconv of this CTA's halves: warps 8-9 keys, 10-11 values ==
-        setmaxnreg_dec112();
+        setmaxnreg_dec80();
         const bool is_v = warp >= 10;
         const int v = threadIdx.x - (is_v ? 320 : 256);
         const int bar_id = is_v ? 2 : 1;
@@ -155,7 +155,7 @@ attn_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
             mbar_arrive_cta(&ready[st], 0);
         }
     } else {
-        setmaxnreg_dec48();
+        setmaxnreg_dec64();
         if (warp == 12 && lane == 0) {
             // ============================================== TMA producer ==
             tma_prefetch_desc(&tm_q);

@@ -21,13 +21,15 @@ struct PrefillArgs {
     int B, T, Hq, Hkv, window, d_max, nqb;
 };
 
-// Register split per warpgroup: 2 x 128 softmax threads at 176, 128 sconv
-// threads at 112, 128 producer/MMA/idle threads at 48: 45056 + 14336 + 6144 =
+// Register split per warpgroup: 2 x 128 softmax threads at 184, 128 sconv
+// threads at 80, 128 producer/MMA/idle threads at 64: 47104 + 10240 + 8192 =
 // 65536 = 512 threads x the 128 registers the kernels launch with (ptxas
 // reports 128), so the increase never waits on registers that do not exist.
-INK_DEV void setmaxnreg_inc176() { asm volatile("setmaxnreg.inc.sync.aligned.u32 176;"); }
-INK_DEV void setmaxnreg_dec112() { asm volatile("setmaxnreg.dec.sync.aligned.u32 112;"); }
-INK_DEV void setmaxnreg_dec48() { asm volatile("setmaxnreg.dec.sync.aligned.u32 48;"); }
+// (At 48 the MMA issuer spills, and its loads from local memory sit on the
+// S -> softmax -> P -> MMA chain.)
+INK_DEV void setmaxnreg_inc184() { asm volatile("setmaxnreg.inc.sync.aligned.u32 184;"); }
+INK_DEV void setmaxnreg_dec80() { asm volatile("setmaxnreg.dec.sync.aligned.u32 80;"); }
+INK_DEV void setmaxnreg_dec64() { asm volatile("setmaxnreg.dec.sync.aligned.u32 64;"); }
 
 // Taps of 8 consecutive channels starting at `wg` ([C, 4] fp32), as channel
 // pairs: w[tap][p] = (w[2p][tap], w[2p+1][tap]).
