@@ -6,6 +6,8 @@
 
 #include "common.cuh"
 
+#include <type_traits>
+
 namespace inkling {
 
 constexpr int kQRows = 256;     // query rows per CTA: two 128-row tiles
@@ -155,20 +157,27 @@ INK_DEV void softmax_role(const PrefillArgs &a, float *bias_sm, uint64_t *s_full
         const float4 *rp = (const float4 *)(bb + sh * kBiasCopy + (o_rd - sh));
         float x[128];
         const int dist0 = i - j0;  // distance of key j0 + c is dist0 - c
-        const bool full = (dist0 - 127 >= 0) && (W <= 0 || dist0 < W) && (j0 + 127 < T);
+        // the keys this row may see in this tile are the columns cmin..cmax:
+        // dist0 - c >= 0, dist0 - c < W (when windowed) and j0 + c < T
+        const int cmax = min(min(127, dist0), T - 1 - j0);
+        const int cmin = (W > 0) ? max(0, dist0 - W + 1) : 0;
+        const bool full = cmin == 0 && cmax == 127;
         // logits and row max, 32 columns at a time: the 8 bias loads of a batch
         // are issued together, and 8 independent 3-input max chains run
-        // alongside
+        // alongside.  Rows of a partial tile take the same paired FMAs and then
+        // mask the columns outside cmin..cmax (a compare of the unrolled column
+        // index against two bounds), in a separate copy of the loop so that
+        // full rows pay nothing for it.
         float m8[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
+        const f32x2 sc2 = pk2(scale, scale);
+        auto logits = [&](auto masked) {
 #pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
-            float4 b4[8];
+            for (int cb = 0; cb < 4; ++cb) {
+                float4 b4[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) b4[j] = rp[cb * 8 + j];
-            if (full) {
-                const f32x2 sc2 = pk2(scale, scale);
+                for (int j = 0; j < 8; ++j) b4[j] = rp[cb * 8 + j];
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const int c = 32 * cb + 4 * j;
@@ -178,24 +187,19 @@ INK_DEV void softmax_role(const PrefillArgs &a, float *bias_sm, uint64_t *s_full
                                            sc2, pk2(b4[j].z, b4[j].w));
                     upk2(xa, x[c], x[c + 1]);
                     upk2(xb, x[c + 2], x[c + 3]);
-                    m8[j] = max3f(max3f(m8[j], x[c], x[c + 1]), x[c + 2], x[c + 3]);
-                }
-            } else {
+                    if (decltype(masked)::value) {
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const float bq[4] = {b4[j].x, b4[j].y, b4[j].z, b4[j].w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int c = 32 * cb + 4 * j + e;
-                        const int dist = dist0 - c;
-                        const bool allowed = dist >= 0 && (W <= 0 || dist < W) && (j0 + c < T);
-                        x[c] = allowed ? fmaf(__uint_as_float(sr[c]), scale, bq[e]) : -INFINITY;
+                        for (int e = 0; e < 4; ++e)
+                            x[c + e] = (c + e >= cmin && c + e <= cmax) ? x[c + e] : -INFINITY;
                     }
-                    const int c = 32 * cb + 4 * j;
                     m8[j] = max3f(max3f(m8[j], x[c], x[c + 1]), x[c + 2], x[c + 3]);
                 }
             }
-        }
+        };
+        if (full)
+            logits(std::false_type{});
+        else
+            logits(std::true_type{});
         const float mx =
             fmaxf(max3f(m8[0], m8[1], m8[2]), max3f(max3f(m8[3], m8[4], m8[5]), m8[6], m8[7]));
         // lazy rescale: move the reference only when the max grows by > tau

@@ -60,6 +60,25 @@ def test_prefill_ragged_and_masks(oracle_mod, B, T, Hq, Hkv, W, D_max):
     assert_parity(out, ref, f"B{B} T{T} Hq{Hq} Hkv{Hkv} W{W} D{D_max}")
 
 
+@pytest.mark.parametrize("B,T,Hq,Hkv,W", [
+    (1, 2560, 32, 4, 0),      # 160 CTA pairs: more than fit on the GPU at once
+    (2, 2500, 32, 4, 1000),   # 320 pairs, ragged tail, window not a multiple of a tile
+])
+def test_prefill_several_waves_all_rows(oracle_mod, B, T, Hq, Hkv, W):
+    """More (head pair, query block) CTA pairs than fit on the GPU at once, with
+    full and partial (window-edge, diagonal, ragged-tail) tiles; every row and
+    its log-sum-exp are compared."""
+    need_gpu()
+    spec = scaled(WORKLOADS["prefill_swa_b4_t8192"], B=B, T=T, Hq=Hq, Hkv=Hkv, window=W,
+                  D_max=3000, seed=11 + W)
+    t = make_prefill(spec)
+    out, lse = _run(t, W)
+    ref, ref_lse = _oracle_all(oracle_mod, t, W)
+    assert_parity(out, ref, f"B{B} T{T} Hq{Hq} Hkv{Hkv} W{W}")
+    got_lse = lse.permute(0, 2, 1).cpu().numpy().reshape(-1)
+    np.testing.assert_allclose(got_lse, ref_lse, rtol=0, atol=2e-3)
+
+
 def test_prefill_window_at_least_T_equals_full():
     need_gpu()
     spec = scaled(WORKLOADS["prefill_tiny_b1_t256"], T=600, Hq=8, Hkv=2, D_max=700, seed=5)
