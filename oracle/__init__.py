@@ -64,6 +64,7 @@ def _load():
             lib.oracle_prefill_rows.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, P, I,
                                                 P, P, P, P]
             lib.oracle_decode_rows.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P, I, P, P]
+            lib.oracle_decode_mq_rows.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, P, I, P, P]
             _lib = lib
     return _lib
 
@@ -211,4 +212,32 @@ def decode_rows(q, k_cache, v_cache, block_table, seq_lens, bias, window, D_max,
     _load().oracle_decode_rows(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(bt), _ptr(sl),
                                _ptr(bias), Hq, Hkv, d, bt.shape[1], int(window), int(D_max),
                                _ptr(pairs), n, _ptr(out), _ptr(lse))
+    return out, lse
+
+
+def decode_mq_rows(q, k_cache, v_cache, block_table, seq_lens, bias, window, D_max, rows=None):
+    """Multi-token decode: query qi of sequence s sits at position L_s - q_len + qi.
+
+    q [S, q_len, Hq, d] bf16 bits; caches [num_blocks, Hkv, 128, d] bf16 bits;
+    rows int array [n, 3] of (s, qi, h), None for all in [S, q_len, Hq] order.
+    Returns (out [n, d] fp64, lse [n] fp64)."""
+    q, k_cache, v_cache = _u16(q), _u16(k_cache), _u16(v_cache)
+    S, Q, Hq, d = q.shape
+    Hkv = k_cache.shape[1]
+    assert k_cache.shape[2] == 128
+    bt = _i32(block_table)
+    sl = _i32(seq_lens)
+    assert (sl >= Q).all(), "every sequence holds its q_len new tokens"
+    bias = _f32(bias)
+    assert bias.shape == (Hq, D_max + 1)
+    if rows is None:
+        ss, qq, hh = np.meshgrid(np.arange(S), np.arange(Q), np.arange(Hq), indexing="ij")
+        rows = np.stack([ss.ravel(), qq.ravel(), hh.ravel()], axis=1)
+    rows = _i32(rows).reshape(-1, 3)
+    n = rows.shape[0]
+    out = np.empty((n, d), np.float64)
+    lse = np.empty((n,), np.float64)
+    _load().oracle_decode_mq_rows(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(bt), _ptr(sl),
+                                  _ptr(bias), Hq, Hkv, d, bt.shape[1], int(window), int(D_max),
+                                  Q, _ptr(rows), n, _ptr(out), _ptr(lse))
     return out, lse

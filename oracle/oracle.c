@@ -313,3 +313,29 @@ void oracle_decode_rows(const uint16_t *q, const uint16_t *k_cache, const uint16
         if (lse) lse[r] = l;
     }
 }
+
+/* Multi-token decode (draft tokens of speculative decoding / multi-token
+ * prediction, vLLM Recipes "thinkingmachines/Inkling", Overview, MTP bullet:
+ * up to 9 tokens per forward step).  A sequence of length L (the q_len new
+ * tokens already appended to the cache) has queries q [S, q_len, Hq, d];
+ * query qi sits at position i = L - q_len + qi and sees keys j <= i (inside
+ * the window), with the bias at distance i - j.  rows holds (s, qi, h)
+ * triples; out and lse are per row. */
+void oracle_decode_mq_rows(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                           const int32_t *block_table, const int32_t *seq_lens,
+                           const float *bias, int64_t Hq, int64_t Hkv, int64_t d,
+                           int64_t max_blocks, int64_t window, int64_t D_max, int64_t q_len,
+                           const int32_t *rows, int64_t n_rows, double *out, double *lse)
+{
+    const int64_t G = Hq / Hkv;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n_rows; ++r) {
+        int64_t s = rows[3 * r], qi = rows[3 * r + 1], h = rows[3 * r + 2];
+        int64_t L = seq_lens[s];
+        paged_ctx ctx = {k_cache, v_cache, block_table + s * max_blocks, h / G, Hkv, d};
+        double l = attn_row(q + ((s * q_len + qi) * Hq + h) * d, paged_key, paged_val, &ctx,
+                            L - q_len + qi, L, window, d, bias + h * (D_max + 1), D_max,
+                            out + r * d);
+        if (lse) lse[r] = l;
+    }
+}

@@ -410,3 +410,55 @@ def test_decode_equals_prefill_last_row_and_block_order(oracle_mod):
                                           W, D_max)
         np.testing.assert_allclose(out, ref, rtol=0, atol=1e-13)
         np.testing.assert_allclose(lse, ref_lse, rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("Q,W,D_max", [(1, 0, 300), (3, 100, 200), (9, 0, 40), (9, 7, 300)])
+def test_decode_mq_equals_prefill_rows(oracle_mod, Q, W, D_max):
+    # q_len draft tokens appended at the end of a sequence of length T: query
+    # qi sits at T - Q + qi, sees keys up to itself (inside the window) and
+    # gets the bias at its own distance; this must equal the prefill rows of
+    # the same positions, for any placement of the blocks in the pool, with the
+    # cache holding the prefill's post-sconv keys and values
+    S, Hq, Hkv, d = 2, 4, 2, 128
+    T = 261
+    C = Hkv * d
+    q = rand_bf16((S, T, Hq, d))
+    k, v = rand_bf16((S, T, Hkv, d)), rand_bf16((S, T, Hkv, d))
+    wk = rng.standard_normal((C, 4)).astype(np.float32) * 0.5
+    wv = rng.standard_normal((C, 4)).astype(np.float32) * 0.5
+    b = rng.standard_normal((Hq, D_max + 1)).astype(np.float32)
+    rows = np.array([[s, h, i] for s in range(S) for i in range(T - Q, T) for h in range(Hq)],
+                    np.int32)
+    ref, ref_lse, kc_all, vc_all = oracle_mod.prefill_rows(q, k, v, wk, wv, b, W, D_max)
+    ref = ref.reshape(S, T, Hq, d)
+    ref_lse = ref_lse.reshape(S, T, Hq)
+    kc_all = kc_all.reshape(S, T, Hkv, d)
+    vc_all = vc_all.reshape(S, T, Hkv, d)
+    nb = 3
+    perm = rng.permutation(S * nb + 4).astype(np.int32)[: S * nb]
+    bt = perm.reshape(S, nb)
+    kc = rand_bf16((S * nb + 4, Hkv, 128, d))     # unused slots hold noise
+    vc = rand_bf16((S * nb + 4, Hkv, 128, d))
+    for s in range(S):
+        for j in range(T):
+            kc[bt[s, j // 128], :, j % 128] = kc_all[s, j]
+            vc[bt[s, j // 128], :, j % 128] = vc_all[s, j]
+    out, lse = oracle_mod.decode_mq_rows(q[:, T - Q:], kc, vc, bt, np.full(S, T, np.int32), b,
+                                         W, D_max)
+    np.testing.assert_allclose(out.reshape(S, Q, Hq, d), ref[:, T - Q:], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse.reshape(S, Q, Hq), ref_lse[:, T - Q:], rtol=0, atol=1e-12)
+    assert rows.shape[0] == S * Q * Hq
+
+
+def test_decode_mq_single_token_equals_decode(oracle_mod):
+    S, Hq, Hkv, d, W, D_max = 3, 8, 2, 128, 50, 64
+    nb = 2
+    lens = np.array([1, 130, 256], np.int32)
+    q = rand_bf16((S, Hq, d))
+    kc, vc = rand_bf16((S * nb, Hkv, 128, d)), rand_bf16((S * nb, Hkv, 128, d))
+    bt = rng.permutation(S * nb).astype(np.int32).reshape(S, nb)
+    b = rng.standard_normal((Hq, D_max + 1)).astype(np.float32)
+    one, lse1 = oracle_mod.decode_rows(q, kc, vc, bt, lens, b, W, D_max)
+    mq, lse2 = oracle_mod.decode_mq_rows(q[:, None], kc, vc, bt, lens, b, W, D_max)
+    np.testing.assert_array_equal(mq, one)
+    np.testing.assert_array_equal(lse2, lse1)
