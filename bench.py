@@ -186,7 +186,8 @@ class DecodeStep:
         self.splits = ink.decode_num_splits(t["q"], t["k_cache"], t["v_cache"],
                                             t["block_table"], t["seq_lens"], t["bias"],
                                             window=spec.window)
-        nbytes = max(16, ink.decode_workspace_bytes(spec.S, spec.Hq, self.splits))
+        rows = spec.S * (t["q"].shape[1] if t["q"].dim() == 4 else 1)  # (sequence, token) rows
+        nbytes = max(16, ink.decode_workspace_bytes(rows, spec.Hq, self.splits))
         self.ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
         self.kv_bytes = kv_bytes_read(spec, t["seq_lens"].cpu())
         self.launches = 2 + (1 if self.splits > 1 else 0)
@@ -345,17 +346,23 @@ def oracle_decode_sample(spec, seconds, seed=0):
     bt, sl = t["block_table"].numpy(), t["seq_lens"].numpy()
     W = sub.window
     done_bytes, total_t, nseq = 0, 0.0, 0
+    Q = sub.n_new
     for s in range(sub.S):
-        pairs = np.array([[s, h] for h in range(sub.Hq)], np.int32)
         t0 = time.perf_counter()
         oracle.sconv_append(u(t["k_new"])[s:s + 1], ks[s:s + 1], t["w_k"].numpy(), kc,
                             bt[s:s + 1], sl[s:s + 1])
         oracle.sconv_append(u(t["v_new"])[s:s + 1], vs[s:s + 1], t["w_v"].numpy(), vc,
                             bt[s:s + 1], sl[s:s + 1])
-        oracle.decode_rows(u(t["q"]), kc, vc, bt, sl, t["bias"].numpy(), W, sub.D_max, pairs)
+        if Q == 1:
+            pairs = np.array([[s, h] for h in range(sub.Hq)], np.int32)
+            oracle.decode_rows(u(t["q"]), kc, vc, bt, sl, t["bias"].numpy(), W, sub.D_max, pairs)
+        else:
+            rows = np.array([[s, qi, h] for qi in range(Q) for h in range(sub.Hq)], np.int32)
+            oracle.decode_mq_rows(u(t["q"]), kc, vc, bt, sl, t["bias"].numpy(), W, sub.D_max,
+                                  rows)
         total_t += time.perf_counter() - t0
         L = int(sl[s])
-        done_bytes += (min(L, W) if W > 0 else L) * sub.Hkv * sub.d * 4
+        done_bytes += (min(L, W + Q - 1) if W > 0 else L) * sub.Hkv * sub.d * 4
         nseq += 1
         if total_t >= seconds:
             break

@@ -151,24 +151,34 @@ typedef struct {
 inkling_status inkling_attn_prefill(const inkling_prefill_params *p, inkling_stream_t stream);
 
 /* --------------------------------------------------------------------------
- * inkling_attn_decode — single-token decode over the paged cache, split-KV.
+ * inkling_attn_decode — decode over the paged cache, split-KV.
  *
  * For sequence s with length L = seq_lens[s], the query q[s] sits at position
  * L-1 and attends to positions max(0, L-window) .. L-1 (0 .. L-1 when
  * window = 0), read through block_table, with the same logits as prefill.
+ *
+ * Multi-token decode (q_len >= 2): the draft tokens of speculative decoding /
+ * multi-token prediction (vLLM Recipes "thinkingmachines/Inkling", Overview,
+ * MTP bullet: 8 chained MTP heads, up to 9 tokens per forward step).  The
+ * q_len newest tokens of each sequence, already appended to the cache, are
+ * all queries: q [S, q_len, Hq, d]; query qi sits at position
+ * i = L - q_len + qi and sees keys j <= i (and i - j < window), with the bias
+ * at distance i - j, so the draft tokens are causal among themselves.
+ * out [S, q_len, Hq, d], lse [S, q_len, Hq].  Needs seq_lens[s] >= q_len
+ * (else INKLING_STATUS_BAD_LENGTH) and G * q_len <= 80.
  * The key range of every sequence is cut into num_splits parts that run on
  * separate thread blocks; their partial (max, sum, unnormalised output)
  * triples go to the caller's workspace and a second kernel merges them.
  * -------------------------------------------------------------------------- */
 typedef struct {
-    const void *q;               /* device [S, Hq, d] bf16 */
+    const void *q;               /* device [S, Hq, d] bf16 ([S, q_len, Hq, d] if q_len >= 2) */
     const void *k_cache;         /* device [num_blocks, Hkv, 128, d] bf16, post-sconv */
     const void *v_cache;         /* device [num_blocks, Hkv, 128, d] bf16, post-sconv */
     const int32_t *block_table;  /* device [S, max_blocks] */
     const int32_t *seq_lens;     /* device [S], each in [1, max_blocks*128] */
     const float *bias;           /* device [Hq, d_max+1] fp32 */
-    void *out;                   /* device [S, Hq, d] bf16 */
-    float *lse;                  /* device [S, Hq] fp32 or NULL */
+    void *out;                   /* device [S, Hq, d] bf16 ([S, q_len, Hq, d] if q_len >= 2) */
+    float *lse;                  /* device [S, Hq] fp32 ([S, q_len, Hq]) or NULL */
     int32_t *status;             /* device int32 or NULL */
     int32_t num_seqs;            /* S >= 0 */
     int32_t num_q_heads;         /* Hq = G * Hkv with 1 <= G <= 8 */
@@ -179,10 +189,12 @@ typedef struct {
     int32_t window;              /* 0 = full */
     int32_t d_max;               /* >= 0 */
     int32_t num_splits;          /* 0 = choose from the SM count, else 1..1024 */
+    int32_t q_len;               /* query tokens per sequence: 0 or 1 = one, 2..10 = multi-token */
 } inkling_decode_params;
 
 /* Workspace bytes inkling_attn_decode needs for num_splits splits (pass the
  * value the call will use, or the result of inkling_attn_decode_num_splits).
+ * For multi-token decode pass num_seqs * q_len as num_seqs.
  * Returns 0 for invalid arguments. */
 size_t inkling_attn_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
                                            int32_t num_splits);

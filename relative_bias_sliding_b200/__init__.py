@@ -7,6 +7,7 @@ libinkling.so (hand-written CUDA, C ABI in include/inkling.h); ``binding``
 marshals torch tensors into it and ``inputs`` draws seeded synthetic inputs.
 """
 from .binding import (  # noqa: F401
+    InklingError,
     attn_decode,
     attn_decode_static,
     attn_prefill,
@@ -17,4 +18,4 @@ from .binding import (  # noqa: F401
 )
 
 __all__ = ["attn_prefill", "attn_decode", "attn_decode_static", "sconv_kv", "decode_num_splits",
-           "decode_workspace_bytes", "load_library"]
+           "decode_workspace_bytes", "load_library", "InklingError"]

@@ -57,7 +57,7 @@ class DecodeParams(ctypes.Structure):
                 ("seq_lens", _P), ("bias", _P), ("out", _P), ("lse", _P), ("status", _P),
                 ("num_seqs", _I), ("num_q_heads", _I), ("num_kv_heads", _I), ("head_dim", _I),
                 ("max_blocks", _I), ("num_blocks", _I), ("window", _I), ("d_max", _I),
-                ("num_splits", _I)]
+                ("num_splits", _I), ("q_len", _I)]
 
 
 class InklingError(RuntimeError):
@@ -191,9 +191,17 @@ def attn_prefill(q, k_raw, v_raw, w_k, w_v, bias, window=0, out=None, lse=None, 
 
 def _decode_params(q, k_cache, v_cache, block_table, seq_lens, bias, window, out, lse, status,
                    num_splits):
+    """q [S, Hq, d] (one token per sequence) or [S, q_len, Hq, d] (the q_len
+    newest tokens of each sequence, multi-token decode)."""
     bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
-    _dev(q, bf, "q", 3)
-    S, Hq, d = q.shape
+    if not isinstance(q, torch.Tensor) or q.dim() not in (3, 4):
+        raise ValueError("q must be [S, Hq, d] or [S, q_len, Hq, d]")
+    _dev(q, bf, "q", q.dim())
+    if q.dim() == 3:
+        S, Hq, d = q.shape
+        Q = 1
+    else:
+        S, Q, Hq, d = q.shape
     _dev(k_cache, bf, "k_cache", 4), _dev(v_cache, bf, "v_cache", 4)
     if k_cache.shape != v_cache.shape or k_cache.shape[2] != BLOCK_SIZE or k_cache.shape[3] != d:
         raise ValueError("caches must be [num_blocks, Hkv, 128, d] and equal")
@@ -204,18 +212,18 @@ def _decode_params(q, k_cache, v_cache, block_table, seq_lens, bias, window, out
     _dev(bias, f32, "bias", 2)
     if bias.shape[0] != Hq:
         raise ValueError("bias must be [Hq, d_max+1]")
-    _dev(out, bf, "out", 3)
+    _dev(out, bf, "out", q.dim())
     if out.shape != q.shape:
         raise ValueError("out must match q")
     if lse is not None:
-        _dev(lse, f32, "lse", 2)
-        if lse.shape != (S, Hq):
-            raise ValueError("lse must be [S, Hq]")
+        _dev(lse, f32, "lse", q.dim() - 1)
+        if lse.shape != q.shape[:-1]:
+            raise ValueError("lse must be q.shape[:-1]")
     _dev(status, i32, "status")
     return DecodeParams(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
                         _ptr(bias), _ptr(out), _ptr(lse), _ptr(status), S, Hq, Hkv, d,
                         block_table.shape[1], k_cache.shape[0], int(window), bias.shape[1] - 1,
-                        int(num_splits))
+                        int(num_splits), Q if q.dim() == 4 else 0)
 
 
 def decode_num_splits(q, k_cache, v_cache, block_table, seq_lens, bias, window=0, num_splits=0):
@@ -236,8 +244,10 @@ def decode_workspace_bytes(num_seqs, num_q_heads, num_splits):
 
 def attn_decode(q, k_cache, v_cache, block_table, seq_lens, bias, window=0, out=None, lse=None,
                 workspace=None, num_splits=0, status=None, stream=None):
-    """Single-token paged decode; returns ``out`` [S, Hq, d] bf16.  ``workspace``
-    (uint8 CUDA tensor) is allocated here by torch when not given."""
+    """Paged decode; returns ``out`` shaped like ``q``: [S, Hq, d] for one token
+    per sequence, [S, q_len, Hq, d] for multi-token decode (the q_len newest
+    tokens of each sequence, causal among themselves).  ``workspace`` (uint8
+    CUDA tensor) is allocated here by torch when not given."""
     if out is None:
         out = torch.empty_like(q)
     p = _decode_params(q, k_cache, v_cache, block_table, seq_lens, bias, window, out, lse, status,
@@ -246,7 +256,8 @@ def attn_decode(q, k_cache, v_cache, block_table, seq_lens, bias, window=0, out=
     splits = lib.inkling_attn_decode_num_splits(ctypes.byref(p))
     if splits <= 0:
         _check(INKLING_ERR_INVALID if not lib.inkling_last_error() else INKLING_ERR_INVALID)
-    need = lib.inkling_attn_decode_workspace_bytes(p.num_seqs, p.num_q_heads, splits)
+    need = lib.inkling_attn_decode_workspace_bytes(p.num_seqs * max(p.q_len, 1), p.num_q_heads,
+                                                   splits)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     _dev(workspace, torch.uint8, "workspace")
@@ -257,9 +268,10 @@ def attn_decode(q, k_cache, v_cache, block_table, seq_lens, bias, window=0, out=
 
 def attn_decode_static(q, k_cache, v_cache, block_table, seq_lens, bias, window=0, out=None,
                        lse=None, num_splits=0, status=None, stream=None):
-    """Single-token paged decode that uses the library's own 8 MiB scratch for
-    the split partials instead of a workspace (for callers that cannot
-    allocate).  Calls must not overlap on the GPU; returns ``out``."""
+    """Paged decode (one or q_len tokens per sequence, as attn_decode) that uses
+    the library's own 8 MiB scratch for the split partials instead of a
+    workspace (for callers that cannot allocate).  Calls must not overlap on
+    the GPU; returns ``out``."""
     if out is None:
         out = torch.empty_like(q)
     p = _decode_params(q, k_cache, v_cache, block_table, seq_lens, bias, window, out, lse, status,

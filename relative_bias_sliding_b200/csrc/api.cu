@@ -97,6 +97,11 @@ inkling_status check_device(int *num_sms) {
     return INKLING_OK;
 }
 
+// sequences x query tokens: the rows of split partials
+static int32_t decode_rows(const inkling_decode_params &p) {
+    return p.num_seqs * (p.q_len > 1 ? p.q_len : 1);
+}
+
 int decode_splits(const inkling_decode_params &p, int num_sms) {
     if (p.num_splits > 0) return p.num_splits;
     const long max_keys = (long)p.max_blocks * 128;
@@ -131,6 +136,12 @@ inkling_status validate_decode(const inkling_decode_params *p) {
     if (p->window < 0 || p->d_max < 0) return fail(INKLING_ERR_INVALID, "window and d_max must be >= 0");
     if (p->num_splits < 0 || p->num_splits > 1024)
         return fail(INKLING_ERR_INVALID, "num_splits must be in [0, 1024]");
+    if (p->q_len < 0) return fail(INKLING_ERR_INVALID, "q_len must be >= 0");
+    if (p->q_len > 1 && (p->num_q_heads / p->num_kv_heads) * p->q_len > 80)
+        return fail(INKLING_ERR_UNSUPPORTED,
+                    "multi-token decode supports (query heads per kv head) * q_len <= 80");
+    if ((long)p->num_seqs * (p->q_len > 1 ? p->q_len : 1) * p->num_q_heads >= (1L << 31))
+        return fail(INKLING_ERR_UNSUPPORTED, "num_seqs * q_len * num_q_heads exceeds 2^31");
     if (p->num_seqs == 0) return INKLING_OK;
     if (!p->q || !p->k_cache || !p->v_cache || !p->block_table || !p->seq_lens || !p->bias || !p->out)
         return fail(INKLING_ERR_INVALID, "a required pointer is NULL");
@@ -284,16 +295,16 @@ inkling_status inkling_attn_decode_static(const inkling_decode_params *p, inklin
     cudaError_t e = decode_static_scratch(&scratch, &cap);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the decode scratch");
     int splits = decode_splits(*p, sms);
-    if (inkling_attn_decode_workspace_bytes(p->num_seqs, p->num_q_heads, splits) > cap) {
+    const int32_t rows = decode_rows(*p);
+    if (inkling_attn_decode_workspace_bytes(rows, p->num_q_heads, splits) > cap) {
         if (p->num_splits > 0)
             return fail(INKLING_ERR_INVALID,
                         "num_splits %d needs %zu bytes of partials; the static scratch holds %zu "
                         "(use fewer splits, or inkling_attn_decode with a workspace)",
-                        splits, inkling_attn_decode_workspace_bytes(p->num_seqs, p->num_q_heads, splits),
+                        splits, inkling_attn_decode_workspace_bytes(rows, p->num_q_heads, splits),
                         cap);
         // automatic split count: the largest that fits (1 needs no scratch)
-        while (splits > 1 &&
-               inkling_attn_decode_workspace_bytes(p->num_seqs, p->num_q_heads, splits) > cap)
+        while (splits > 1 && inkling_attn_decode_workspace_bytes(rows, p->num_q_heads, splits) > cap)
             --splits;
     }
     return decode_with(p, splits, scratch, cap, stream);
@@ -303,7 +314,7 @@ static inkling_status decode_with(const inkling_decode_params *p, int splits, vo
                                   size_t workspace_bytes, inkling_stream_t stream) {
     inkling_status st;
     if (splits > 1) {
-        const size_t need = inkling_attn_decode_workspace_bytes(p->num_seqs, p->num_q_heads, splits);
+        const size_t need = inkling_attn_decode_workspace_bytes(decode_rows(*p), p->num_q_heads, splits);
         if (!workspace || workspace_bytes < need)
             return fail(INKLING_ERR_INVALID, "workspace of %zu bytes given, %zu needed for %d splits",
                         workspace_bytes, need, splits);

@@ -83,6 +83,10 @@ WORKLOADS = {
                                     1 << 20, 0.5, 4),
     "decode_full_1m_b8": DecodeSpec("decode_full_1m_b8", 8, 1 << 20, 1 << 20, 64, 8, 128, 0,
                                     1 << 20, 0.5, 4),
+    # sliding-window decode verifying 9 draft tokens per sequence (multi-token
+    # prediction: up to 9 tokens per forward step)
+    "decode_mtp9_swa_s64": DecodeSpec("decode_mtp9_swa_s64", 64, 1024, 32768, 64, 8, 128, 4096,
+                                      4096, 1.0, 3, n_new=9),
     # smaller cuts of the same workloads for profiler captures (still larger
     # than L2, a few GB on the device at most)
     "prefill_swa_b1_t8192": PrefillSpec("prefill_swa_b1_t8192", 1, 8192, 64, 8, 128, 4096,
@@ -138,7 +142,9 @@ def make_decode(spec: DecodeSpec, device="cpu", extra_blocks: int = 0):
     g = _generator(device, spec.seed)
     S, Hq, Hkv, d, n_new = spec.S, spec.Hq, spec.Hkv, spec.d, spec.n_new
     C = Hkv * d
-    q = _normal_bf16(g, (S, Hq, d), device)
+    # one query per sequence, or the n_new newest tokens all as queries
+    # (multi-token decode: the draft tokens of speculative decoding)
+    q = _normal_bf16(g, (S, Hq, d) if n_new == 1 else (S, n_new, Hq, d), device)
     k_new = _normal_bf16(g, (S, n_new, Hkv, d), device)
     v_new = _normal_bf16(g, (S, n_new, Hkv, d), device)
     w_k = torch.randn((C, 4), generator=g, device=device, dtype=torch.float32) * 0.5
@@ -170,10 +176,11 @@ def make_decode(spec: DecodeSpec, device="cpu", extra_blocks: int = 0):
 
 
 def kv_bytes_read(spec: DecodeSpec, seq_lens) -> int:
-    """Post-sconv K+V bytes inside each sequence's window or context."""
+    """Post-sconv K+V bytes inside each sequence's window or context (for
+    n_new query tokens, the union of their windows: W + n_new - 1 keys)."""
     W = spec.window
     tot = 0
     for L in seq_lens.tolist():
-        n = min(L, W) if W > 0 else L
+        n = min(L, W + spec.n_new - 1) if W > 0 else L
         tot += n
     return tot * spec.Hkv * spec.d * 2 * 2
