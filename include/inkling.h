@@ -107,7 +107,7 @@ typedef struct {
     const int32_t *seq_lens;     /* device [S], lengths after the append, >= n_new */
     int32_t *status;             /* device int32 or NULL */
     int32_t num_seqs;            /* S >= 0 (0 = nothing to do) */
-    int32_t n_new;               /* new tokens per sequence, 1..64 */
+    int32_t n_new;               /* new tokens per sequence, 1..2^20 (a decode step or a prefill chunk) */
     int32_t num_kv_heads;        /* Hkv >= 1 */
     int32_t head_dim;            /* d, must be 128 */
     int32_t max_blocks;          /* columns of block_table */
@@ -149,6 +149,59 @@ typedef struct {
 } inkling_prefill_params;
 
 inkling_status inkling_attn_prefill(const inkling_prefill_params *p, inkling_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * inkling_attn_prefill_paged — chunked prefill over the paged cache.
+ *
+ * A chunk of new tokens per sequence (variable lengths, rows packed): the
+ * chunk's queries attend to the whole sequence so far through the paged cache
+ * of post-sconv keys and values (vLLM Recipes "thinkingmachines/Inkling",
+ * Overview: "Attention", and "Short convolution", whose cache is managed like
+ * a sliding-window layer's KV cache; Client Usage: 128-token blocks).
+ *
+ * Call order for one chunk:
+ *  1. inkling_sconv_kv with n_new = the chunk length.  It convolves the
+ *     chunk's raw keys and values, continuing from the rolling 3-token state,
+ *     and writes them into the cache.
+ *  2. This call.
+ *
+ * Sequence s has n_s = cu_q[s+1] - cu_q[s] new tokens and length
+ * L_s = seq_lens[s] after them.  Its query r (packed row cu_q[s] + r) sits at
+ * position L_s - n_s + r and sees keys j <= that position, inside the window,
+ * with the bias at distance position - j.  The rows equal rows
+ * L_s - n_s .. L_s - 1 of inkling_attn_prefill on the whole sequence.
+ *
+ * Sequences with n_s = 0 produce nothing.
+ *  - n_s > max_q, n_s < 0 or L_s < n_s: INKLING_STATUS_BAD_LENGTH.  Rows
+ *    past max_q are not written.
+ *  - A block id outside [0, num_blocks): INKLING_STATUS_BAD_BLOCK (block 0
+ *    is read instead).
+ * -------------------------------------------------------------------------- */
+typedef struct {
+    const void *q;               /* device [total_q, Hq, d] bf16, rows of all sequences packed */
+    const int32_t *cu_q;         /* device [S+1] nondecreasing row offsets, cu_q[0] = 0 */
+    const void *k_cache;         /* device [num_blocks, Hkv, 128, d] bf16, post-sconv */
+    const void *v_cache;         /* device [num_blocks, Hkv, 128, d] bf16, post-sconv */
+    const int32_t *block_table;  /* device [S, max_blocks] */
+    const int32_t *seq_lens;     /* device [S] lengths including the new tokens */
+    const float *bias;           /* device [Hq, d_max+1] fp32 */
+    void *out;                   /* device [total_q, Hq, d] bf16 */
+    float *lse;                  /* device [total_q, Hq] fp32 natural-log row logsumexp, or NULL */
+    int32_t *status;             /* device int32 or NULL */
+    int32_t num_seqs;            /* S >= 0 */
+    int32_t total_q;             /* rows of q / out (= cu_q[S]) */
+    int32_t max_q;               /* >= every n_s (sizes the grid) */
+    int32_t num_q_heads;         /* Hq, a multiple of Hkv */
+    int32_t num_kv_heads;        /* Hkv >= 1 */
+    int32_t head_dim;            /* d, must be 128 */
+    int32_t max_blocks;          /* columns of block_table */
+    int32_t num_blocks;          /* blocks in the pool */
+    int32_t window;              /* 0 = full causal, else keys with i-j < window */
+    int32_t d_max;               /* >= 0 */
+} inkling_prefill_paged_params;
+
+inkling_status inkling_attn_prefill_paged(const inkling_prefill_paged_params *p,
+                                          inkling_stream_t stream);
 
 /* --------------------------------------------------------------------------
  * inkling_attn_decode — decode over the paged cache, split-KV.

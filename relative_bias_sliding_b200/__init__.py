@@ -11,11 +11,12 @@ from .binding import (  # noqa: F401
     attn_decode,
     attn_decode_static,
     attn_prefill,
+    attn_prefill_paged,
     decode_num_splits,
     decode_workspace_bytes,
     load_library,
     sconv_kv,
 )
 
-__all__ = ["attn_prefill", "attn_decode", "attn_decode_static", "sconv_kv", "decode_num_splits",
+__all__ = ["attn_prefill", "attn_prefill_paged", "attn_decode", "attn_decode_static", "sconv_kv", "decode_num_splits",
            "decode_workspace_bytes", "load_library", "InklingError"]

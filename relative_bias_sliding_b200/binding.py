@@ -28,6 +28,7 @@ EXPORTED = (
     "inkling_selftest_wait_timeout",
     "inkling_sconv_kv",
     "inkling_attn_prefill",
+    "inkling_attn_prefill_paged",
     "inkling_attn_decode_workspace_bytes",
     "inkling_attn_decode_num_splits",
     "inkling_attn_decode",
@@ -50,6 +51,14 @@ class PrefillParams(ctypes.Structure):
                 ("out", _P), ("lse", _P), ("status", _P), ("batch", _I), ("seq_len", _I),
                 ("num_q_heads", _I), ("num_kv_heads", _I), ("head_dim", _I), ("window", _I),
                 ("d_max", _I)]
+
+
+class PrefillPagedParams(ctypes.Structure):
+    _fields_ = [("q", _P), ("cu_q", _P), ("k_cache", _P), ("v_cache", _P), ("block_table", _P),
+                ("seq_lens", _P), ("bias", _P), ("out", _P), ("lse", _P), ("status", _P),
+                ("num_seqs", _I), ("total_q", _I), ("max_q", _I), ("num_q_heads", _I),
+                ("num_kv_heads", _I), ("head_dim", _I), ("max_blocks", _I), ("num_blocks", _I),
+                ("window", _I), ("d_max", _I)]
 
 
 class DecodeParams(ctypes.Structure):
@@ -87,6 +96,8 @@ def load_library(path: str = LIB_PATH):
         lib.inkling_sconv_kv.restype = ctypes.c_int
         lib.inkling_attn_prefill.argtypes = [ctypes.POINTER(PrefillParams), _P]
         lib.inkling_attn_prefill.restype = ctypes.c_int
+        lib.inkling_attn_prefill_paged.argtypes = [ctypes.POINTER(PrefillPagedParams), _P]
+        lib.inkling_attn_prefill_paged.restype = ctypes.c_int
         lib.inkling_attn_decode_workspace_bytes.argtypes = [_I, _I, _I]
         lib.inkling_attn_decode_workspace_bytes.restype = ctypes.c_size_t
         lib.inkling_attn_decode_num_splits.argtypes = [ctypes.POINTER(DecodeParams)]
@@ -186,6 +197,50 @@ def attn_prefill(q, k_raw, v_raw, w_k, w_v, bias, window=0, out=None, lse=None, 
     p = PrefillParams(_ptr(q), _ptr(k_raw), _ptr(v_raw), _ptr(w_k), _ptr(w_v), _ptr(bias),
                       _ptr(out), _ptr(lse), _ptr(status), B, T, Hq, Hkv, d, int(window), d_max)
     _check(load_library().inkling_attn_prefill(ctypes.byref(p), _stream(stream)))
+    return out
+
+
+def attn_prefill_paged(q, cu_q, k_cache, v_cache, block_table, seq_lens, bias, window=0,
+                       max_q=None, out=None, lse=None, status=None, stream=None):
+    """Chunked prefill over the paged cache (see inkling.h): ``q`` [total_q, Hq, d]
+    packs the new tokens of every sequence (rows cu_q[s] .. cu_q[s+1]-1), whose
+    keys and values sconv_kv has already appended; ``seq_lens`` are the lengths
+    including them.  ``max_q`` bounds every chunk length (read from ``cu_q``
+    with a device sync when not given).  Returns ``out`` [total_q, Hq, d]."""
+    bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    _dev(q, bf, "q", 3)
+    total_q, Hq, d = q.shape
+    _dev(cu_q, i32, "cu_q", 1)
+    S = cu_q.shape[0] - 1
+    if S < 0:
+        raise ValueError("cu_q must have num_seqs + 1 entries")
+    _dev(k_cache, bf, "k_cache", 4), _dev(v_cache, bf, "v_cache", 4)
+    if k_cache.shape != v_cache.shape or k_cache.shape[2] != BLOCK_SIZE or k_cache.shape[3] != d:
+        raise ValueError("caches must be [num_blocks, Hkv, 128, d] and equal")
+    Hkv = k_cache.shape[1]
+    _dev(block_table, i32, "block_table", 2), _dev(seq_lens, i32, "seq_lens", 1)
+    if block_table.shape[0] != S or seq_lens.shape[0] != S:
+        raise ValueError("block_table / seq_lens must have num_seqs rows")
+    _dev(bias, f32, "bias", 2)
+    if bias.shape[0] != Hq:
+        raise ValueError("bias must be [Hq, d_max+1]")
+    if out is None:
+        out = torch.empty_like(q)
+    _dev(out, bf, "out", 3)
+    if out.shape != q.shape:
+        raise ValueError("out must match q")
+    if lse is not None:
+        _dev(lse, f32, "lse", 2)
+        if lse.shape != (total_q, Hq):
+            raise ValueError("lse must be [total_q, Hq]")
+    _dev(status, i32, "status")
+    if max_q is None:
+        max_q = int((cu_q[1:] - cu_q[:-1]).max().item()) if S > 0 else 0
+    p = PrefillPagedParams(_ptr(q), _ptr(cu_q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                           _ptr(seq_lens), _ptr(bias), _ptr(out), _ptr(lse), _ptr(status), S,
+                           total_q, int(max_q), Hq, Hkv, d, block_table.shape[1],
+                           k_cache.shape[0], int(window), bias.shape[1] - 1)
+    _check(load_library().inkling_attn_prefill_paged(ctypes.byref(p), _stream(stream)))
     return out
 
 

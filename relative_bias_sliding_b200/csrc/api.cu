@@ -12,6 +12,9 @@ namespace inkling {
 cudaError_t launch_sconv_kv(const inkling_sconv_params &p, cudaStream_t stream);
 cudaError_t launch_attn_prefill(const inkling_prefill_params &p, const CUtensorMap *maps,
                                 cudaStream_t stream);
+cudaError_t launch_attn_prefill_paged(const inkling_prefill_paged_params &p, const CUtensorMap &tm_q,
+                                      const CUtensorMap &tm_k, const CUtensorMap &tm_v,
+                                      cudaStream_t stream);
 cudaError_t launch_attn_prefill_pair(const inkling_prefill_params &p, const CUtensorMap *maps,
                                      cudaStream_t stream);
 cudaError_t launch_attn_decode(const inkling_decode_params &p, int splits, void *workspace,
@@ -179,7 +182,10 @@ inkling_status inkling_sconv_kv(const inkling_sconv_params *p, inkling_stream_t 
         return fail(INKLING_ERR_INVALID, "num_seqs must be >= 0, num_kv_heads >= 1");
     if (p->head_dim != INKLING_HEAD_DIM)
         return fail(INKLING_ERR_UNSUPPORTED, "head_dim %d (only 128 is implemented)", p->head_dim);
-    if (p->n_new < 1 || p->n_new > 64) return fail(INKLING_ERR_INVALID, "n_new must be in [1, 64]");
+    if (p->n_new < 1 || p->n_new > (1 << 20))
+        return fail(INKLING_ERR_INVALID, "n_new must be in [1, 2^20]");
+    if ((long)p->num_seqs * p->n_new * p->num_kv_heads * 16 * 2 >= (1L << 40))
+        return fail(INKLING_ERR_UNSUPPORTED, "too many tokens in one append");
     if (p->max_blocks < 1 || p->num_blocks < 1)
         return fail(INKLING_ERR_INVALID, "max_blocks and num_blocks must be >= 1");
     if ((long)p->max_blocks * 128 > (1L << 30))
@@ -253,6 +259,60 @@ inkling_status inkling_attn_prefill(const inkling_prefill_params *p, inkling_str
     }
     cudaError_t e = launch_attn_prefill(*p, maps, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "attn_prefill launch");
+    return INKLING_OK;
+}
+
+inkling_status inkling_attn_prefill_paged(const inkling_prefill_paged_params *p,
+                                          inkling_stream_t stream) {
+    g_err[0] = 0;
+    if (!p) return fail(INKLING_ERR_INVALID, "params is NULL");
+    if (p->num_seqs < 0 || p->total_q < 0 || p->max_q < 0 || p->num_q_heads < 1 ||
+        p->num_kv_heads < 1)
+        return fail(INKLING_ERR_INVALID, "sizes must be >= 0 and head counts >= 1");
+    if (p->head_dim != INKLING_HEAD_DIM)
+        return fail(INKLING_ERR_UNSUPPORTED, "head_dim %d (only 128 is implemented)", p->head_dim);
+    if (p->num_q_heads % p->num_kv_heads)
+        return fail(INKLING_ERR_INVALID, "num_q_heads %% num_kv_heads != 0");
+    if (p->max_blocks < 1 || p->num_blocks < 1)
+        return fail(INKLING_ERR_INVALID, "max_blocks and num_blocks must be >= 1");
+    if ((long)p->max_blocks * 128 > (1L << 30))
+        return fail(INKLING_ERR_UNSUPPORTED, "max_blocks * 128 exceeds 2^30 tokens");
+    if ((long)p->num_blocks * p->num_kv_heads * 128 >= (1L << 31))
+        return fail(INKLING_ERR_UNSUPPORTED, "cache pool rows exceed 2^31");
+    if ((long)p->total_q * p->num_q_heads >= (1L << 31))
+        return fail(INKLING_ERR_UNSUPPORTED, "total_q * num_q_heads exceeds 2^31");
+    if (p->window < 0 || p->d_max < 0) return fail(INKLING_ERR_INVALID, "window and d_max must be >= 0");
+    if (p->num_seqs == 0 || p->total_q == 0 || p->max_q == 0) return INKLING_OK;
+    if ((long)p->num_seqs * p->num_q_heads * ((p->max_q + 255) / 256) >= (1L << 31))
+        return fail(INKLING_ERR_UNSUPPORTED, "grid too large");
+    if (!p->q || !p->cu_q || !p->k_cache || !p->v_cache || !p->block_table || !p->seq_lens ||
+        !p->bias || !p->out)
+        return fail(INKLING_ERR_INVALID, "a required pointer is NULL");
+    if (!aligned16(p->q) || !aligned16(p->k_cache) || !aligned16(p->v_cache) || !aligned16(p->out))
+        return fail(INKLING_ERR_INVALID, "q, caches and out must be 16-byte aligned");
+    if (((uintptr_t)p->bias & 3u) != 0) return fail(INKLING_ERR_INVALID, "bias must be 4-byte aligned");
+    inkling_status st = check_device(nullptr);
+    if (st != INKLING_OK) return st;
+    CUtensorMap tm_q, tm_k, tm_v;
+    {
+        // q [total_q, Hq, 128] seen as (d, head, row): one box = 128 rows x 64 d of one head
+        const cuuint64_t Hq = (cuuint64_t)p->num_q_heads;
+        cuuint64_t dims[3] = {128, Hq, (cuuint64_t)p->total_q};
+        cuuint64_t str[2] = {256, Hq * 256};
+        cuuint32_t box[3] = {64, 1, 128};
+        if ((st = make_map(&tm_q, p->q, 3, dims, str, box)) != INKLING_OK) return st;
+    }
+    {
+        // caches as (d, rows): one box = one 128-token (block, kv head) x 64 d
+        const cuuint64_t rows = (cuuint64_t)p->num_blocks * p->num_kv_heads * 128;
+        cuuint64_t dims[2] = {128, rows};
+        cuuint64_t str[1] = {256};
+        cuuint32_t box[2] = {64, 128};
+        if ((st = make_map(&tm_k, p->k_cache, 2, dims, str, box)) != INKLING_OK) return st;
+        if ((st = make_map(&tm_v, p->v_cache, 2, dims, str, box)) != INKLING_OK) return st;
+    }
+    cudaError_t e = launch_attn_prefill_paged(*p, tm_q, tm_k, tm_v, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "attn_prefill_paged launch");
     return INKLING_OK;
 }
 

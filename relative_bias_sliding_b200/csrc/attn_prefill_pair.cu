@@ -117,11 +117,12 @@ attn_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int t = warp >> 2;
         if (ok[t])
             softmax_role(a, (float *)(smem + PBIAS) + t * 2 * kBiasBuf, &bar[S_FULL], &bar[O_DONE],
-                         abort_flag, tbase, t, b, h, r0[t], lo[t], hi[t], 3 + t,
-                         smem + PQ + t * 32768, &tm_out, [&](int tt) {
+                         abort_flag, tbase, t, h, r0[t], a.T, lo[t], hi[t], 3 + t,
+                         [&](int tt) {
                              __syncwarp();
                              if (lane == 0) mbar_arrive_cta_relaxed(&bar[P_FULL + tt], 0);
-                         });
+                         },
+                         TmaStoreEpilogue{a, smem + PQ + t * 32768, &tm_out, b, h, r0[t], 3 + t});
     } else if (warp < 12) {
         // ==================== sconv of this CTA's halves: warps 8-9 keys, 10-11 values ==
         setmaxnreg_dec80();

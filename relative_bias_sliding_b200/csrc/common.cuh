@@ -109,6 +109,13 @@ INK_DEV void tma_load_2d(void *dst, const CUtensorMap *m, uint64_t *bar, int x, 
         : "memory");
 }
 
+INK_DEV void tma_load_3d(void *dst, const CUtensorMap *m, uint64_t *bar, int x, int y, int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(m), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
 INK_DEV void tma_load_4d(void *dst, const CUtensorMap *m, uint64_t *bar, int x, int y, int z,
                          int w) {
     asm volatile(

@@ -95,31 +95,84 @@ INK_DEV void sconv_rows(uint32_t tile, uint32_t hist, uint32_t half_bytes, const
     }
 }
 
+// Normalised output of one query row: O / l from tensor memory as 16 chunks of
+// 8 bf16 (16 bytes), handed to store(c, chunk) for c = 0..15.
+template <class Store>
+INK_DEV void emit_row(uint32_t o_col, float l, Store store) {
+    const float inv = (l > 0.f) ? 1.f / l : 0.f;
+#pragma unroll
+    for (int cb = 0; cb < 4; ++cb) {
+        uint32_t orr[32];
+        tmem_ld32(o_col + cb * 32, orr);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+            uint4 v;
+            v.x = pack_bf16(__uint_as_float(orr[q4 * 8 + 0]) * inv, __uint_as_float(orr[q4 * 8 + 1]) * inv);
+            v.y = pack_bf16(__uint_as_float(orr[q4 * 8 + 2]) * inv, __uint_as_float(orr[q4 * 8 + 3]) * inv);
+            v.z = pack_bf16(__uint_as_float(orr[q4 * 8 + 4]) * inv, __uint_as_float(orr[q4 * 8 + 5]) * inv);
+            v.w = pack_bf16(__uint_as_float(orr[q4 * 8 + 6]) * inv, __uint_as_float(orr[q4 * 8 + 7]) * inv);
+            store(cb * 4 + q4, v);
+        }
+    }
+}
+
+// Epilogue of the dense prefill: the normalised bf16 O tile is staged in
+// `stage` (the query tile's shared-memory buffer, free once the last QK^T of
+// the tile has completed) in the same 128-byte-swizzled layout, and one thread
+// writes it with two bulk tensor stores through `tm_out`, a [B, T, Hq, 128]
+// map (rows past the sequence end are clipped).  Every thread of the group
+// calls it (the named barrier counts 128).
+struct TmaStoreEpilogue {
+    const PrefillArgs &a;
+    uint8_t *stage;
+    const CUtensorMap *tm_out;
+    int b, h, r0, bar_id;
+    INK_DEV void operator()(bool have_o, int u, int i, float l, float m_ref, uint32_t o_col,
+                            volatile int *abort_flag) const {
+        if (have_o) {
+            emit_row(o_col, l, [&](int c, uint4 v) {
+                *(uint4 *)(stage + (c >> 3) * 16384 + u * 128 + (((c & 7) ^ (u & 7)) << 4)) = v;
+            });
+            if (a.lse && i < a.T)
+                a.lse[((long)b * a.Hq + h) * a.T + i] = (l > 0.f) ? m_ref + __logf(l) : -INFINITY;
+            fence_proxy_async_smem();
+        }
+        // every warp of the group reaches this barrier (have_o is uniform per warp)
+        named_bar_sync(bar_id, 128);
+        if (u == 0 && have_o && !*abort_flag) {
+            tma_store_4d(tm_out, stage, 0, r0, h, b);
+            tma_store_4d(tm_out, stage + 16384, 64, r0, h, b);
+            bulk_commit_group();
+            bulk_wait_all();
+        }
+    }
+};
+
 // Softmax of one 128-row query tile (the calling warpgroup; thread = row =
-// TMEM lane), over key tiles lo..hi, then the epilogue.  S lives in TMEM
-// columns [128t, 128t+128), O in [256+128t, ...); P (bf16) is written over the
-// first 64 columns of S.  `signal_p(t)` is called by every thread once its P
-// and O updates are complete and fenced; it must tell the MMA issuer.
-// `bias_sm` holds this tile's two bias-diagonal buffers; `bar_id` is a named
-// barrier private to this warpgroup.
-// The epilogue stages the normalised bf16 O tile in `stage` (the query tile's
-// shared-memory buffer, free once the last QK^T of the tile has completed) in
-// the same 128-byte-swizzled layout, and one thread writes it with two bulk
-// tensor stores through `tm_out` (rows past the sequence end are clipped).
-template <class SignalP>
+// TMEM lane), over key tiles lo..hi, then the epilogue.  Row u of the tile is
+// the query at sequence position pos0 + u; keys exist at positions
+// 0 .. key_end-1.  S lives in TMEM columns [128t, 128t+128), O in
+// [256+128t, ...); P (bf16) is written over the first 64 columns of S.
+// `signal_p(t)` is called by every thread once its P and O updates are
+// complete and fenced; it must tell the MMA issuer.  `bias_sm` holds this
+// tile's two bias-diagonal buffers; `bar_id` is a named barrier private to
+// this warpgroup.  At the end every thread calls
+// epilogue(have_o, u, pos0 + u, l, m_ref, o_col, abort_flag).
+template <class SignalP, class Epilogue>
 INK_DEV void softmax_role(const PrefillArgs &a, float *bias_sm, uint64_t *s_full, uint64_t *o_done,
-                          volatile int *abort_flag, uint32_t tbase, int t, int b, int h, int r0,
-                          int lo, int hi, int bar_id, uint8_t *stage, const CUtensorMap *tm_out,
-                          SignalP signal_p) {
+                          volatile int *abort_flag, uint32_t tbase, int t, int h, int pos0,
+                          int key_end, int lo, int hi, int bar_id, SignalP signal_p,
+                          const Epilogue &epilogue) {
     const int u = threadIdx.x & 127;
     const uint32_t tl = tbase + ((uint32_t)(((threadIdx.x >> 5) & 3) * 32) << 16);
     const uint32_t s_col = tl + t * 128, o_col = tl + 256 + t * 128;
-    const int i = r0 + u;
+    const int i = pos0 + u;
     const float scale = 0.08838834764831845f;  // 1/sqrt(128)
     const float kLog2e = 1.4426950408889634f;
     const float kTau = 5.545177444479562f;     // 8 ln 2
     const float *bias_h = a.bias + (long)h * (a.d_max + 1);
-    const int W = a.window, Dm = a.d_max, T = a.T;
+    const int W = a.window, Dm = a.d_max, T = key_end;
     float m_ref = -INFINITY, l = 0.f;
     const int o_rd = 127 - u, sh = o_rd & 3;  // this row's start in the staged diagonal
     bool dead = false;
@@ -127,12 +180,12 @@ INK_DEV void softmax_role(const PrefillArgs &a, float *bias_sm, uint64_t *s_full
     for (int n = lo; n <= hi; ++n, ++k) {
         const int j0 = n * 128;
         // Stage the bias diagonal of this (query tile, key tile) pair:
-        // R[q] = bias[h, clamp(top - q, 0, d_max)], q = 0..254, top = r0 - j0 + 127,
+        // R[q] = bias[h, clamp(top - q, 0, d_max)], q = 0..254, top = pos0 - j0 + 127,
         // as 4 copies shifted by 0..3 floats so that row u reads R[127-u+c],
         // c = 0..127, with aligned 16-byte loads.  Double-buffered by tile parity.
         float *bb = bias_sm + (k & 1) * kBiasBuf;
         {
-            const int top = r0 - j0 + 127;
+            const int top = pos0 - j0 + 127;
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const int q = 2 * u + e;
@@ -248,39 +301,9 @@ INK_DEV void softmax_role(const PrefillArgs &a, float *bias_sm, uint64_t *s_full
         tc_fence_before();
         signal_p(t);
     }
-    // epilogue: O / l -> bf16, staged in shared memory, one bulk store per half
     const bool have_o = !dead && mbar_wait_warp(&o_done[t], 0, abort_flag, a.status);
-    if (have_o) {
-        tc_fence_after();
-        const float inv = (l > 0.f) ? 1.f / l : 0.f;
-#pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
-            uint32_t orr[32];
-            tmem_ld32(o_col + cb * 32, orr);
-            tmem_wait_ld();
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                uint4 v;
-                v.x = pack_bf16(__uint_as_float(orr[q4 * 8 + 0]) * inv, __uint_as_float(orr[q4 * 8 + 1]) * inv);
-                v.y = pack_bf16(__uint_as_float(orr[q4 * 8 + 2]) * inv, __uint_as_float(orr[q4 * 8 + 3]) * inv);
-                v.z = pack_bf16(__uint_as_float(orr[q4 * 8 + 4]) * inv, __uint_as_float(orr[q4 * 8 + 5]) * inv);
-                v.w = pack_bf16(__uint_as_float(orr[q4 * 8 + 6]) * inv, __uint_as_float(orr[q4 * 8 + 7]) * inv);
-                const int c = cb * 4 + q4;  // 16-byte chunk of the 256-byte row
-                *(uint4 *)(stage + (c >> 3) * 16384 + u * 128 + (((c & 7) ^ (u & 7)) << 4)) = v;
-            }
-        }
-        if (a.lse && i < T)
-            a.lse[((long)b * a.Hq + h) * T + i] = (l > 0.f) ? m_ref + __logf(l) : -INFINITY;
-        fence_proxy_async_smem();
-    }
-    // every warp of the group reaches this barrier (have_o is uniform per warp)
-    named_bar_sync(bar_id, 128);
-    if (u == 0 && have_o && !*abort_flag) {
-        tma_store_4d(tm_out, stage, 0, r0, h, b);
-        tma_store_4d(tm_out, stage + 16384, 64, r0, h, b);
-        bulk_commit_group();
-        bulk_wait_all();
-    }
+    if (have_o) tc_fence_after();
+    epilogue(have_o, u, i, l, m_ref, o_col, abort_flag);
 }
 
 }  // namespace inkling

@@ -1,15 +1,20 @@
 // sconv_kv.cu — decode-side sconv append (vLLM Recipes "thinkingmachines/
 // Inkling", Overview, "Short convolution": window-4 sconv on keys and values,
-// its state managed like the KV cache of a sliding-window layer).
-//
-// One thread owns 8 consecutive channels of one sequence's keys or values:
-// it reads the 3 raw history tokens from the state, convolves each new token,
-// writes the bf16 result to the token's slot in the paged cache
-// (block_table[s, pos/128], slot pos%128) and stores the last 3 raw tokens
-// back as the new state.  Memory-bound: 16-byte loads and stores, one pass.
+// its state managed like the KV cache of a sliding-window layer).  The same
+// call appends one decode token, a few draft tokens or a whole prefill chunk.
 #include "common.cuh"
 
 namespace inkling {
+
+// One thread owns 8 consecutive channels of one sequence's keys or values and
+// a run of up to kRun consecutive new tokens: it reads the 3 raw tokens before
+// its run (from the state for the first run, from the new tokens otherwise),
+// convolves each token of the run and writes the bf16 result to the token's
+// slot in the paged cache (block_table[s, pos/128], slot pos%128).  The thread
+// of the first run also writes the new state, the last 3 raw tokens of
+// (old state, new tokens), after it has read the old one; no other thread
+// touches the state.  Memory-bound: 16-byte loads and stores, one pass.
+constexpr int kRun = 32;
 
 __global__ void __launch_bounds__(128)
 sconv_kv_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new,
@@ -19,11 +24,13 @@ sconv_kv_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new
                 const int32_t *__restrict__ block_table, const int32_t *__restrict__ seq_lens,
                 int32_t *status, int S, int n_new, int Hkv, int max_blocks, int num_blocks) {
     const int chunks = Hkv * 16;  // 8-channel chunks per token (C = Hkv*128)
+    const int runs = (n_new + kRun - 1) / kRun;
     const long gid = (long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (gid >= (long)S * 2 * chunks) return;
+    if (gid >= (long)S * 2 * chunks * runs) return;
     const int chunk = (int)(gid % chunks);
     const int which = (int)((gid / chunks) & 1);  // 0 = keys, 1 = values
-    const int s = (int)(gid / (2 * chunks));
+    const int run = (int)((gid / (2 * chunks)) % runs);
+    const int s = (int)(gid / (2L * chunks * runs));
 
     const uint4 *xin = which ? v_new : k_new;
     const float4 *wt = which ? w_v : w_k;
@@ -41,18 +48,28 @@ sconv_kv_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new
         const float4 t = wt[chunk * 8 + e];
         w[e][0] = t.x; w[e][1] = t.y; w[e][2] = t.z; w[e][3] = t.w;
     }
-    // state [S, 3, C] bf16 = per token `chunks` uint4
+    // raw history: state [S, 3, C] (oldest first) or new tokens [S, n_new, C]
+    const int t0 = run * kRun, t1 = min(n_new, t0 + kRun);
+    auto new_tok = [&](int t) { return xin[((long)s * n_new + t) * chunks + chunk]; };
+    uint4 r3, r2, r1;
+    if (run == 0) {
+        r3 = state[((long)s * 3 + 0) * chunks + chunk];
+        r2 = state[((long)s * 3 + 1) * chunks + chunk];
+        r1 = state[((long)s * 3 + 2) * chunks + chunk];
+    } else {
+        r3 = new_tok(t0 - 3);
+        r2 = new_tok(t0 - 2);
+        r1 = new_tok(t0 - 1);
+    }
+    const uint4 s3 = r3, s2 = r2, s1 = r1;  // the old state, for the first run
     float h3[8], h2[8], h1[8];
-    uint4 r3 = state[((long)s * 3 + 0) * chunks + chunk];
-    uint4 r2 = state[((long)s * 3 + 1) * chunks + chunk];
-    uint4 r1 = state[((long)s * 3 + 2) * chunks + chunk];
     unpack8(r3, h3);
     unpack8(r2, h2);
     unpack8(r1, h1);
 
     const int kvh = chunk >> 4, e16 = chunk & 15;  // kv head, 16-byte column in the row
-    for (int t = 0; t < n_new; ++t) {
-        const uint4 raw = xin[((long)s * n_new + t) * chunks + chunk];
+    for (int t = t0; t < t1; ++t) {
+        const uint4 raw = new_tok(t);
         float x[8];
         unpack8(raw, x);
         const uint4 y = sconv8(w, h3, h2, h1, x);
@@ -63,17 +80,25 @@ sconv_kv_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new
         } else {
             cache[(((long)blk * Hkv + kvh) * 128 + (pos & 127)) * 16 + e16] = y;
         }
-        r3 = r2; r2 = r1; r1 = raw;
 #pragma unroll
         for (int e = 0; e < 8; ++e) { h3[e] = h2[e]; h2[e] = h1[e]; h1[e] = x[e]; }
     }
-    state[((long)s * 3 + 0) * chunks + chunk] = r3;
-    state[((long)s * 3 + 1) * chunks + chunk] = r2;
-    state[((long)s * 3 + 2) * chunks + chunk] = r1;
+    if (run == 0) {
+        // new state: the last 3 of (old state s3 s2 s1, new tokens 0..n_new-1)
+        uint4 ns[3];
+#pragma unroll
+        for (int m = 0; m < 3; ++m) {
+            const int idx = n_new + m;  // index in the concatenated stream of 3 + n_new
+            ns[m] = idx >= 3 ? new_tok(idx - 3) : (idx == 0 ? s3 : (idx == 1 ? s2 : s1));
+        }
+#pragma unroll
+        for (int m = 0; m < 3; ++m) state[((long)s * 3 + m) * chunks + chunk] = ns[m];
+    }
 }
 
 cudaError_t launch_sconv_kv(const inkling_sconv_params &p, cudaStream_t stream) {
-    const long threads = (long)p.num_seqs * 2 * p.num_kv_heads * 16;
+    const long runs = (p.n_new + kRun - 1) / kRun;
+    const long threads = (long)p.num_seqs * 2 * p.num_kv_heads * 16 * runs;
     if (threads == 0) return cudaSuccess;
     const int block = 128;
     const long grid = (threads + block - 1) / block;

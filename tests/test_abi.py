@@ -45,10 +45,13 @@ def test_struct_layouts_match_header(tmp_path):
 #include "{HEADER}"
 #define F(S, m) printf(#S " " #m " %zu\\n", offsetof(S, m));
 int main(void) {{
-  printf("sconv %zu\\nprefill %zu\\ndecode %zu\\n", sizeof(inkling_sconv_params),
-         sizeof(inkling_prefill_params), sizeof(inkling_decode_params));
+  printf("sconv %zu\\nprefill %zu\\ndecode %zu\\npaged %zu\\n", sizeof(inkling_sconv_params),
+         sizeof(inkling_prefill_params), sizeof(inkling_decode_params),
+         sizeof(inkling_prefill_paged_params));
   F(inkling_sconv_params, num_blocks) F(inkling_prefill_params, d_max)
   F(inkling_decode_params, num_splits) F(inkling_decode_params, status)
+  F(inkling_decode_params, q_len) F(inkling_prefill_paged_params, cu_q)
+  F(inkling_prefill_paged_params, max_q) F(inkling_prefill_paged_params, d_max)
   return 0;
 }}""")
     exe = tmp_path / "sizes"
@@ -62,6 +65,12 @@ int main(void) {{
     assert int(out["inkling_prefill_params d_max"]) == binding.PrefillParams.d_max.offset
     assert int(out["inkling_decode_params num_splits"]) == binding.DecodeParams.num_splits.offset
     assert int(out["inkling_decode_params status"]) == binding.DecodeParams.status.offset
+    assert int(out["inkling_decode_params q_len"]) == binding.DecodeParams.q_len.offset
+    P = binding.PrefillPagedParams
+    assert int(out["paged"]) == ctypes.sizeof(P)
+    assert int(out["inkling_prefill_paged_params cu_q"]) == P.cu_q.offset
+    assert int(out["inkling_prefill_paged_params max_q"]) == P.max_q.offset
+    assert int(out["inkling_prefill_paged_params d_max"]) == P.d_max.offset
 
 
 def test_workspace_bytes(lib):
@@ -96,7 +105,7 @@ def test_host_validation_rejects_before_launch(lib):
     assert lib.inkling_attn_decode(ctypes.byref(d), None, 0, None) == binding.INKLING_ERR_INVALID
 
     s = binding.SconvParams()
-    s.num_seqs, s.n_new, s.num_kv_heads, s.head_dim, s.max_blocks, s.num_blocks = 1, 65, 1, 128, 1, 1
+    s.num_seqs, s.n_new, s.num_kv_heads, s.head_dim, s.max_blocks, s.num_blocks = 1, 0, 1, 128, 1, 1
     assert lib.inkling_sconv_kv(ctypes.byref(s), None) == binding.INKLING_ERR_INVALID
     s.n_new = 1
     assert lib.inkling_sconv_kv(ctypes.byref(s), None) == binding.INKLING_ERR_INVALID  # NULLs

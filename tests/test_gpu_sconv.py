@@ -55,8 +55,10 @@ def _run_both(oracle_mod, t):
     return dev, ref
 
 
-@pytest.mark.parametrize("n_new,lens", [(1, [1, 128, 129, 5000, 300]), (3, [3, 130, 256]),
-                                        (7, [7, 200, 1000]), (64, [64, 127, 4096])])
+@pytest.mark.parametrize("n_new,lens", [(1, [1, 128, 129, 5000, 300]), (2, [2, 3, 400]),
+                                        (3, [3, 130, 256]), (7, [7, 200, 1000]),
+                                        (33, [33, 34, 300]), (64, [64, 127, 4096]),
+                                        (1029, [1029, 1300, 4096])])
 def test_sconv_kv_matches_oracle(oracle_mod, n_new, lens):
     need_gpu()
     t = _setup(len(lens), 2, lens, n_new, seed=n_new)
