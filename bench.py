@@ -210,6 +210,33 @@ class DecodeStep:
         self.run_attn(stream)
 
 
+class ChunkStep:
+    """Chunked prefill step: sconv append of every sequence's chunk, then the
+    chunk rows over the paged cache."""
+
+    def __init__(self, spec, device):
+        import torch
+        from relative_bias_sliding_b200.inputs import make_chunk
+        self.spec = spec
+        self.t = make_chunk(spec, device=device)
+        self.out = torch.empty_like(self.t["q"])
+        self.flops = spec.flops
+        self.launches = 2
+
+    def run_append(self, stream=None):
+        import relative_bias_sliding_b200 as ink
+        t = self.t
+        ink.sconv_kv(t["k_new"], t["v_new"], t["w_k"], t["w_v"], t["k_state"], t["v_state"],
+                     t["k_cache"], t["v_cache"], t["block_table"], t["seq_lens"], stream=stream)
+
+    def run_attn(self, stream=None):
+        import relative_bias_sliding_b200 as ink
+        t = self.t
+        ink.attn_prefill_paged(t["q"], t["cu_q"], t["k_cache"], t["v_cache"], t["block_table"],
+                               t["seq_lens"], t["bias"], window=self.spec.window,
+                               max_q=self.spec.chunk, out=self.out, stream=stream)
+
+
 def timed_loop(steps, fns, stream):
     """Run ``steps`` iterations of the callables in order on ``stream``; return
     per-callable mean milliseconds (CUDA events recorded on that stream)."""
@@ -370,6 +397,41 @@ def oracle_decode_sample(spec, seconds, seed=0):
     return done_bytes / total_t / 1e9, desc, oracle.num_threads()
 
 
+def oracle_chunk_sample(spec, seconds, seed=0):
+    """Time the oracle's chunked-prefill step (sconv append of one sequence's
+    chunk, then its chunk rows over the paged cache, all heads) on a bounded
+    sample of rows; returns (TFLOP/s, description, threads)."""
+    import numpy as np
+    import torch
+    import oracle
+    from relative_bias_sliding_b200.inputs import make_chunk, scaled
+    sub = scaled(spec, B=1)
+    t = make_chunk(sub, device="cpu")
+    u = lambda x: x.contiguous().view(torch.int16).numpy().view(np.uint16)
+    kc, vc = u(t["k_cache"]).copy(), u(t["v_cache"]).copy()
+    ks, vs = u(t["k_state"]).copy(), u(t["v_state"]).copy()
+    bt, sl = t["block_table"].numpy(), t["seq_lens"].numpy()
+    n, W = sub.chunk, sub.window
+    q = u(t["q"]).reshape(1, n, sub.Hq, sub.d)
+    t0 = time.perf_counter()
+    oracle.sconv_append(u(t["k_new"]), ks, t["w_k"].numpy(), kc, bt, sl)
+    oracle.sconv_append(u(t["v_new"]), vs, t["w_v"].numpy(), vc, bt, sl)
+    rng = np.random.default_rng(seed)
+    done_flops, rows_done = 0, 0
+    while time.perf_counter() - t0 < seconds:
+        qi = rng.integers(0, n, 16)
+        rows = np.array([[0, r, h] for r in qi for h in range(sub.Hq)], np.int32)
+        oracle.decode_mq_rows(q, kc, vc, bt, sl, t["bias"].numpy(), W, sub.D_max, rows)
+        for r in qi:
+            i = sub.prefix + int(r)
+            done_flops += 4 * sub.d * sub.Hq * (min(i + 1, W) if W > 0 else i + 1)
+        rows_done += len(rows)
+    total_t = time.perf_counter() - t0
+    desc = (f"sconv append of one {n}-token chunk + {rows_done} (row, head) pairs of "
+            f"{spec.name}, {total_t:.1f} s")
+    return done_flops / total_t / 1e12, desc, oracle.num_threads()
+
+
 # ------------------------------------------------------------------ main --
 
 def parse():
@@ -389,7 +451,7 @@ def parse():
 
 
 def run_reference(args):
-    from relative_bias_sliding_b200.inputs import WORKLOADS, PrefillSpec
+    from relative_bias_sliding_b200.inputs import WORKLOADS, PrefillSpec, ChunkSpec
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
@@ -401,6 +463,9 @@ def run_reference(args):
     for k in range(args.warmup + args.steps):
         if isinstance(spec, PrefillSpec):
             v, desc, thr = oracle_prefill_sample(spec, per_step, seed=k)
+            unit = "TFLOP/s"
+        elif isinstance(spec, ChunkSpec):
+            v, desc, thr = oracle_chunk_sample(spec, per_step, seed=k)
             unit = "TFLOP/s"
         else:
             v, desc, thr = oracle_decode_sample(spec, per_step, seed=k)
@@ -421,13 +486,67 @@ def run_reference(args):
     return 0
 
 
+def run_chunk(args, chk, dist, rank, world, local, device):
+    """Bench line of a chunked-prefill workload (device-timed; no e2e leg)."""
+    import torch
+    stream = torch.cuda.Stream(device)
+    fns = [chk.run_append, chk.run_attn]
+    for _ in range(args.warmup):
+        for f in fns:
+            f(stream)
+    stream.synchronize()
+    barrier(dist, device)
+    torch.cuda.synchronize()
+    with ClockSampler(local, args.clocks_log_dir) as clocks:
+        barrier(dist, device)
+        torch.cuda.synchronize()
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        per_fn = timed_loop(args.steps, fns, stream)
+        t_end.record(stream)
+        stream.synchronize()
+        torch.cuda.synchronize()
+        barrier(dist, device)
+    step_ms = t_start.elapsed_time(t_end) / args.steps
+    per_fn = max_over_ranks(dist, per_fn, device)
+    step_ms = max_over_ranks(dist, [step_ms], device)[0]
+    peaks, peak_src = load_peaks()
+    app_ms, attn_ms = per_fn
+    tflops = chk.flops / ((app_ms + attn_ms) * 1e-3) / 1e12 * world
+    kern = chk.flops / (attn_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    line = {"metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "gpu_launches": args.steps * chk.launches,
+            "roofline": {"bound": "tensor", "kernel": "attn_prefill_paged_kernel",
+                         "achieved": kern, "peak": peak, "unit": "TFLOP/s", "frac": kern / peak,
+                         "traffic": MEASURED_TRAFFIC.get(chk.spec.name),
+                         "peak_source": f"{peak_src} bf16_tflops_sustained"},
+            "chunk": {"sconv_append_ms": app_ms, "attn_prefill_paged_ms": attn_ms},
+            "config": {"workload": chk.spec.name, "parallelism": f"replica per GPU x{world}",
+                       "l2": "inputs larger than L2 (q 256 MiB, cache 1 GiB)"},
+            "e2e": None, "clocks": clocks.summary()}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, desc, thr = oracle_chunk_sample(chk.spec, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+                                "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
     import torch
     import relative_bias_sliding_b200 as ink
-    from relative_bias_sliding_b200.inputs import WORKLOADS, PrefillSpec
+    from relative_bias_sliding_b200.inputs import WORKLOADS, PrefillSpec, ChunkSpec
 
     rank, world, local = dist_env()
     if world != args.gpus:
@@ -439,8 +558,11 @@ def main():
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
 
+    chk = None
     if args.workload:
         spec = WORKLOADS[args.workload]
+        if isinstance(spec, ChunkSpec):
+            return run_chunk(args, ChunkStep(spec, device), dist, rank, world, local, device)
         pre = PrefillStep(spec, device) if isinstance(spec, PrefillSpec) else None
         dec = None if pre else DecodeStep(spec, device)
     else:

@@ -65,6 +65,36 @@ class DecodeSpec:
     n_new: int = 1
 
 
+@dataclass(frozen=True)
+class ChunkSpec:
+    """Chunked prefill: B sequences that already hold `prefix` tokens (their
+    post-sconv keys/values in the paged cache, their raw last 3 in the sconv
+    state) receive `chunk` new tokens each, all of them queries."""
+    name: str
+    B: int
+    prefix: int
+    chunk: int
+    Hq: int
+    Hkv: int
+    d: int
+    window: int
+    D_max: int
+    bias_std: float
+    seed: int
+
+    @property
+    def allowed_pairs(self) -> int:
+        """(query, key) pairs of the chunk rows inside the band / window, per (seq, head)."""
+        W, tot = self.window, 0
+        for i in range(self.prefix, self.prefix + self.chunk):
+            tot += min(i + 1, W) if W > 0 else i + 1
+        return tot
+
+    @property
+    def flops(self) -> int:
+        return 4 * self.d * self.Hq * self.B * self.allowed_pairs
+
+
 WORKLOADS = {
     # tiny full-causal prefill, small enough for the oracle on every row
     "prefill_tiny_b1_t256": PrefillSpec("prefill_tiny_b1_t256", 1, 256, 8, 1, 128, 0, 256,
@@ -87,6 +117,10 @@ WORKLOADS = {
     # prediction: up to 9 tokens per forward step)
     "decode_mtp9_swa_s64": DecodeSpec("decode_mtp9_swa_s64", 64, 1024, 32768, 64, 8, 128, 4096,
                                       4096, 1.0, 3, n_new=9),
+    # chunked prefill: 4 sequences with a 6144-token prefix take their last
+    # 2048-token chunk (the sliding-window prefill's shape, cut in chunks)
+    "prefill_chunked_swa_b4_c2048": ChunkSpec("prefill_chunked_swa_b4_c2048", 4, 6144, 2048, 64,
+                                              8, 128, 4096, 4096, 1.0, 5),
     # smaller cuts of the same workloads for profiler captures (still larger
     # than L2, a few GB on the device at most)
     "prefill_swa_b1_t8192": PrefillSpec("prefill_swa_b1_t8192", 1, 8192, 64, 8, 128, 4096,
@@ -184,3 +218,34 @@ def kv_bytes_read(spec: DecodeSpec, seq_lens) -> int:
         n = min(L, W + spec.n_new - 1) if W > 0 else L
         tot += n
     return tot * spec.Hkv * spec.d * 2 * 2
+
+
+def make_chunk(spec: ChunkSpec, device="cpu"):
+    """Chunked-prefill step inputs: packed chunk queries q [B*chunk, Hq, d] with
+    row offsets cu_q, the chunk's raw keys/values [B, chunk, Hkv, d], taps,
+    bias, sconv states, and a paged cache whose prefix slots hold N(0, 1)
+    post-sconv rows (the append overwrites the chunk's slots)."""
+    g = _generator(device, spec.seed)
+    B, Hq, Hkv, d, n = spec.B, spec.Hq, spec.Hkv, spec.d, spec.chunk
+    C = Hkv * d
+    q = _normal_bf16(g, (B * n, Hq, d), device)
+    k_new = _normal_bf16(g, (B, n, Hkv, d), device)
+    v_new = _normal_bf16(g, (B, n, Hkv, d), device)
+    w_k = torch.randn((C, 4), generator=g, device=device, dtype=torch.float32) * 0.5
+    w_v = torch.randn((C, 4), generator=g, device=device, dtype=torch.float32) * 0.5
+    bias = torch.randn((Hq, spec.D_max + 1), generator=g, device=device,
+                       dtype=torch.float32) * spec.bias_std
+    k_state = _normal_bf16(g, (B, 3, C), device)
+    v_state = _normal_bf16(g, (B, 3, C), device)
+    L = spec.prefix + n
+    nb = (L + BLOCK - 1) // BLOCK
+    perm = torch.randperm(B * nb, generator=g, device=device).to(torch.int32)
+    block_table = perm.reshape(B, nb).contiguous()
+    k_cache = _normal_bf16(g, (B * nb, Hkv, BLOCK, d), device)
+    v_cache = _normal_bf16(g, (B * nb, Hkv, BLOCK, d), device)
+    seq_lens = torch.full((B,), L, dtype=torch.int32, device=device)
+    cu_q = torch.arange(0, (B + 1) * n, n, dtype=torch.int32, device=device)
+    return dict(q=q, cu_q=cu_q, k_new=k_new, v_new=v_new, w_k=w_k, w_v=w_v, bias=bias,
+                k_state=k_state, v_state=v_state, seq_lens=seq_lens, block_table=block_table,
+                k_cache=k_cache, v_cache=v_cache)
+

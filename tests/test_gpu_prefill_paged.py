@@ -5,9 +5,9 @@ import numpy as np
 import pytest
 import torch
 
-from conftest import assert_parity, need_gpu, u16
+from conftest import assert_append_close, assert_parity, need_gpu, u16
 import relative_bias_sliding_b200 as ink
-from relative_bias_sliding_b200.inputs import BLOCK
+from relative_bias_sliding_b200.inputs import BLOCK, WORKLOADS as WORKLOADS_CHUNK
 
 pytestmark = pytest.mark.gpu
 
@@ -127,3 +127,43 @@ def test_chunked_prefill_reports_short_length():
                            torch.zeros((Hq, 17), device="cuda"), status=status)
     torch.cuda.synchronize()
     assert status.item() & 4   # INKLING_STATUS_BAD_LENGTH: 10 new tokens, length 5
+
+
+def test_chunked_workload_sampled_rows(oracle_mod):
+    """The chunked-prefill bench workload (4 sequences, 6144-token prefix,
+    2048-token chunk, window 4096): GPU append + paged prefill; sampled
+    (row, head) pairs against the oracle's append + paged attention of the
+    same rows (query r at position prefix + r)."""
+    need_gpu()
+    from relative_bias_sliding_b200.inputs import make_chunk
+    spec = WORKLOADS_CHUNK["prefill_chunked_swa_b4_c2048"]
+    t = make_chunk(spec)
+    host = {k: v.clone() for k, v in t.items()}
+    dev = {k: v.cuda() for k, v in t.items()}
+    ink.sconv_kv(dev["k_new"], dev["v_new"], dev["w_k"], dev["w_v"], dev["k_state"],
+                 dev["v_state"], dev["k_cache"], dev["v_cache"], dev["block_table"],
+                 dev["seq_lens"])
+    out = ink.attn_prefill_paged(dev["q"], dev["cu_q"], dev["k_cache"], dev["v_cache"],
+                                 dev["block_table"], dev["seq_lens"], dev["bias"],
+                                 window=spec.window, max_q=spec.chunk)
+    torch.cuda.synchronize()
+    kc, vc = u16(host["k_cache"]).copy(), u16(host["v_cache"]).copy()
+    ks, vs = u16(host["k_state"]).copy(), u16(host["v_state"]).copy()
+    bt, sl = host["block_table"].numpy(), host["seq_lens"].numpy()
+    oracle_mod.sconv_append(u16(host["k_new"]), ks, host["w_k"].numpy(), kc, bt, sl)
+    oracle_mod.sconv_append(u16(host["v_new"]), vs, host["w_v"].numpy(), vc, bt, sl)
+    # the GPU append (fp32 FMA chain, one bf16 rounding) against the oracle's
+    # (exact sum, one bf16 rounding): within 1 bf16 ulp, or, where the four
+    # tap products cancel, within the fp32 chain's rounding of the terms
+    assert_append_close(u16(dev["k_cache"]), kc)
+    assert_append_close(u16(dev["v_cache"]), vc)
+    rng = np.random.default_rng(0)
+    n = spec.chunk
+    q = u16(host["q"]).reshape(spec.B, n, spec.Hq, 128)
+    rows = np.array([[s, r, h] for s in range(spec.B)
+                     for r in list(rng.integers(0, n, 6)) + [0, n - 1]
+                     for h in rng.integers(0, spec.Hq, 2)], np.int32)
+    ref, _ = oracle_mod.decode_mq_rows(q, kc, vc, bt, sl, host["bias"].numpy(), spec.window,
+                                       spec.D_max, rows)
+    got = out.cpu().reshape(spec.B, n, spec.Hq, 128)[rows[:, 0], rows[:, 1], rows[:, 2]]
+    assert_parity(got, ref, "chunked workload sampled rows")

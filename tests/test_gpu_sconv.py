@@ -3,7 +3,7 @@ import numpy as np
 import pytest
 import torch
 
-from conftest import need_gpu, u16
+from conftest import assert_append_close, need_gpu, u16
 import relative_bias_sliding_b200 as ink
 from relative_bias_sliding_b200.inputs import BLOCK
 
@@ -69,10 +69,10 @@ def test_sconv_kv_matches_oracle(oracle_mod, n_new, lens):
         assert np.array_equal(u16(dev[f"{which}_state"]), st_ref)
         got = u16(dev[f"{which}_cache"]).view(np.int16).astype(np.int32)
         exp = cache_ref.view(np.int16).astype(np.int32)
-        # fp32 FMA chain vs one fp64 rounding: at most 1 bf16 ulp apart, rarely
-        ulps = np.abs(got - exp)
-        assert ulps.max() <= 1, which
-        assert (ulps > 0).mean() < 2e-3, which
+        # fp32 FMA chain vs one rounding of the exact sum: rarely different,
+        # within 1 bf16 ulp or (cancelling taps) the chain's fp32 rounding
+        frac = assert_append_close(u16(dev[f"{which}_cache"]), cache_ref)
+        assert frac < 2e-3, which
         # untouched slots are bit-identical (paging is index work: exact)
         untouched = np.ones(exp.shape, bool)
         bt = t["block_table"].numpy()
