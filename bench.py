@@ -432,6 +432,27 @@ def oracle_chunk_sample(spec, seconds, seed=0):
     return done_flops / total_t / 1e12, desc, oracle.num_threads()
 
 
+def oracle_sconv_out_sample(spec, seconds, seed=0):
+    """Time the oracle's sconv on slices of the output-sconv workload; returns
+    (GB/s of x read + y written, description, threads)."""
+    import numpy as np
+    import torch
+    import oracle
+    from relative_bias_sliding_b200.inputs import make_sconv_out, scaled
+    sub = scaled(spec, B=1, T=min(spec.T, 1024))
+    t = make_sconv_out(sub, device="cpu")
+    x = t["x"].contiguous().view(torch.int16).numpy().view(np.uint16)
+    h = t["state"].contiguous().view(torch.int16).numpy().view(np.uint16)
+    w = t["w"].numpy()
+    t0, n = time.perf_counter(), 0
+    while time.perf_counter() - t0 < seconds or n == 0:
+        oracle.sconv(x, w, h)
+        n += 1
+    dt = time.perf_counter() - t0
+    desc = f"{n} passes over a [1, {sub.T}, {sub.C}] slice of {spec.name}, {dt:.1f} s"
+    return n * sub.bytes_moved / dt / 1e9, desc, oracle.num_threads()
+
+
 # ------------------------------------------------------------------ main --
 
 def parse():
@@ -451,7 +472,7 @@ def parse():
 
 
 def run_reference(args):
-    from relative_bias_sliding_b200.inputs import WORKLOADS, PrefillSpec, ChunkSpec
+    from relative_bias_sliding_b200.inputs import WORKLOADS, PrefillSpec, ChunkSpec, SconvOutSpec
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
@@ -467,6 +488,9 @@ def run_reference(args):
         elif isinstance(spec, ChunkSpec):
             v, desc, thr = oracle_chunk_sample(spec, per_step, seed=k)
             unit = "TFLOP/s"
+        elif isinstance(spec, SconvOutSpec):
+            v, desc, thr = oracle_sconv_out_sample(spec, per_step, seed=k)
+            unit = "GB/s"
         else:
             v, desc, thr = oracle_decode_sample(spec, per_step, seed=k)
             unit = "GB/s"
@@ -540,13 +564,52 @@ def run_chunk(args, chk, dist, rank, world, local, device):
     return 0
 
 
+def run_sconv_out(args, spec, dist, rank, world, local, device):
+    """Bench line of the output sconv (HBM-bound; device-timed, no e2e leg)."""
+    import torch
+    import relative_bias_sliding_b200 as ink
+    from relative_bias_sliding_b200.inputs import make_sconv_out
+    t = make_sconv_out(spec, device=device)
+    y = torch.empty_like(t["x"])
+    stream = torch.cuda.Stream(device)
+    fn = lambda s=None: ink.sconv_out(t["x"], t["w"], t["state"], out=y, stream=s)
+    for _ in range(args.warmup):
+        fn(stream)
+    stream.synchronize()
+    barrier(dist, device)
+    with ClockSampler(local, args.clocks_log_dir) as clocks:
+        torch.cuda.synchronize()
+        ms = timed_loop(args.steps, [fn], stream)[0]
+        barrier(dist, device)
+    ms = max_over_ranks(dist, [ms], device)[0]
+    peaks, peak_src = load_peaks()
+    gbs = spec.bytes_moved / (ms * 1e-3) / 1e9
+    line = {"metric": METRIC, "value": gbs * world, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "gpu_launches": args.steps,
+            "roofline": {"bound": "hbm", "kernel": "sconv_out_kernel", "achieved": gbs,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                         "peak_source": f"{peak_src} hbm_gbs"},
+            "config": {"workload": spec.name, "parallelism": f"replica per GPU x{world}",
+                       "l2": "inputs larger than L2 (x and y 512 MiB each)"},
+            "e2e": None, "clocks": clocks.summary()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
     import torch
     import relative_bias_sliding_b200 as ink
-    from relative_bias_sliding_b200.inputs import WORKLOADS, PrefillSpec, ChunkSpec
+    from relative_bias_sliding_b200.inputs import WORKLOADS, PrefillSpec, ChunkSpec, SconvOutSpec
 
     rank, world, local = dist_env()
     if world != args.gpus:
@@ -561,6 +624,8 @@ def main():
     chk = None
     if args.workload:
         spec = WORKLOADS[args.workload]
+        if isinstance(spec, SconvOutSpec):
+            return run_sconv_out(args, spec, dist, rank, world, local, device)
         if isinstance(spec, ChunkSpec):
             return run_chunk(args, ChunkStep(spec, device), dist, rank, world, local, device)
         pre = PrefillStep(spec, device) if isinstance(spec, PrefillSpec) else None

@@ -151,6 +151,33 @@ typedef struct {
 inkling_status inkling_attn_prefill(const inkling_prefill_params *p, inkling_stream_t stream);
 
 /* --------------------------------------------------------------------------
+ * inkling_sconv_out — the window-4 short convolution on the attention output
+ * (vLLM Recipes "thinkingmachines/Inkling", Overview, "Short convolution":
+ * four sconv modules per layer, on keys, values, output and MoE output).
+ *
+ * y[b,t,c] = sum_{k=0..3} w[c,k] * x[b,t-k,c] for the C channels of the
+ * attention output (C = Hq*128, before the output projection).  The 3 raw
+ * rows before t = 0 come from state (oldest first), or are zero when state is
+ * NULL.  A non-NULL state is then updated in place to the last 3 raw rows of
+ * (old state, x), so a decode step or a prefill chunk continues where the
+ * previous one stopped.
+ *
+ * Arithmetic: fp32, taps applied oldest first with fused multiply-adds, one
+ * bf16 rounding (as inkling_sconv_kv).  x and y must not overlap.
+ * -------------------------------------------------------------------------- */
+typedef struct {
+    const void *x;       /* device [B, T, C] bf16 */
+    const float *w;      /* device [C, 4] fp32 taps (tap 0 = current token) */
+    void *state;         /* device [B, 3, C] bf16 raw history, or NULL (zero history) */
+    void *y;             /* device [B, T, C] bf16 */
+    int32_t batch;       /* B >= 0 */
+    int32_t seq_len;     /* T >= 0 */
+    int32_t channels;    /* C, a positive multiple of 8 */
+} inkling_sconv_out_params;
+
+inkling_status inkling_sconv_out(const inkling_sconv_out_params *p, inkling_stream_t stream);
+
+/* --------------------------------------------------------------------------
  * inkling_attn_prefill_paged — chunked prefill over the paged cache.
  *
  * A chunk of new tokens per sequence (variable lengths, rows packed): the

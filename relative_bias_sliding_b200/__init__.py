@@ -16,7 +16,8 @@ from .binding import (  # noqa: F401
     decode_workspace_bytes,
     load_library,
     sconv_kv,
+    sconv_out,
 )
 
 __all__ = ["attn_prefill", "attn_prefill_paged", "attn_decode", "attn_decode_static", "sconv_kv", "decode_num_splits",
-           "decode_workspace_bytes", "load_library", "InklingError"]
+           "decode_workspace_bytes", "load_library", "InklingError", "sconv_out"]

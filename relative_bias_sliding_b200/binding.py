@@ -27,6 +27,7 @@ EXPORTED = (
     "inkling_version",
     "inkling_selftest_wait_timeout",
     "inkling_sconv_kv",
+    "inkling_sconv_out",
     "inkling_attn_prefill",
     "inkling_attn_prefill_paged",
     "inkling_attn_decode_workspace_bytes",
@@ -51,6 +52,11 @@ class PrefillParams(ctypes.Structure):
                 ("out", _P), ("lse", _P), ("status", _P), ("batch", _I), ("seq_len", _I),
                 ("num_q_heads", _I), ("num_kv_heads", _I), ("head_dim", _I), ("window", _I),
                 ("d_max", _I)]
+
+
+class SconvOutParams(ctypes.Structure):
+    _fields_ = [("x", _P), ("w", _P), ("state", _P), ("y", _P), ("batch", _I), ("seq_len", _I),
+                ("channels", _I)]
 
 
 class PrefillPagedParams(ctypes.Structure):
@@ -96,6 +102,8 @@ def load_library(path: str = LIB_PATH):
         lib.inkling_sconv_kv.restype = ctypes.c_int
         lib.inkling_attn_prefill.argtypes = [ctypes.POINTER(PrefillParams), _P]
         lib.inkling_attn_prefill.restype = ctypes.c_int
+        lib.inkling_sconv_out.argtypes = [ctypes.POINTER(SconvOutParams), _P]
+        lib.inkling_sconv_out.restype = ctypes.c_int
         lib.inkling_attn_prefill_paged.argtypes = [ctypes.POINTER(PrefillPagedParams), _P]
         lib.inkling_attn_prefill_paged.restype = ctypes.c_int
         lib.inkling_attn_decode_workspace_bytes.argtypes = [_I, _I, _I]
@@ -197,6 +205,29 @@ def attn_prefill(q, k_raw, v_raw, w_k, w_v, bias, window=0, out=None, lse=None, 
     p = PrefillParams(_ptr(q), _ptr(k_raw), _ptr(v_raw), _ptr(w_k), _ptr(w_v), _ptr(bias),
                       _ptr(out), _ptr(lse), _ptr(status), B, T, Hq, Hkv, d, int(window), d_max)
     _check(load_library().inkling_attn_prefill(ctypes.byref(p), _stream(stream)))
+    return out
+
+
+def sconv_out(x, w, state=None, out=None, stream=None):
+    """Output sconv: x [B, T, C] bf16 (attention output, C = Hq*128), taps w
+    [C, 4] fp32; state [B, 3, C] bf16 (updated in place) or None for zero
+    history.  Returns y [B, T, C] bf16."""
+    _dev(x, torch.bfloat16, "x", 3)
+    B, T, C = x.shape
+    _dev(w, torch.float32, "w", 2)
+    if w.shape != (C, 4):
+        raise ValueError(f"w must be [{C}, 4]")
+    if state is not None:
+        _dev(state, torch.bfloat16, "state", 3)
+        if state.shape != (B, 3, C):
+            raise ValueError(f"state must be [{B}, 3, {C}]")
+    if out is None:
+        out = torch.empty_like(x)
+    _dev(out, torch.bfloat16, "out", 3)
+    if out.shape != x.shape:
+        raise ValueError("out must match x")
+    p = SconvOutParams(_ptr(x), _ptr(w), _ptr(state), _ptr(out), B, T, C)
+    _check(load_library().inkling_sconv_out(ctypes.byref(p), _stream(stream)))
     return out
 
 

@@ -12,6 +12,7 @@ namespace inkling {
 cudaError_t launch_sconv_kv(const inkling_sconv_params &p, cudaStream_t stream);
 cudaError_t launch_attn_prefill(const inkling_prefill_params &p, const CUtensorMap *maps,
                                 cudaStream_t stream);
+cudaError_t launch_sconv_out(const inkling_sconv_out_params &p, cudaStream_t stream);
 cudaError_t launch_attn_prefill_paged(const inkling_prefill_paged_params &p, const CUtensorMap &tm_q,
                                       const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                                       cudaStream_t stream);
@@ -259,6 +260,29 @@ inkling_status inkling_attn_prefill(const inkling_prefill_params *p, inkling_str
     }
     cudaError_t e = launch_attn_prefill(*p, maps, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "attn_prefill launch");
+    return INKLING_OK;
+}
+
+inkling_status inkling_sconv_out(const inkling_sconv_out_params *p, inkling_stream_t stream) {
+    g_err[0] = 0;
+    if (!p) return fail(INKLING_ERR_INVALID, "params is NULL");
+    if (p->batch < 0 || p->seq_len < 0) return fail(INKLING_ERR_INVALID, "batch and seq_len must be >= 0");
+    if (p->channels < 8 || p->channels % 8)
+        return fail(INKLING_ERR_INVALID, "channels must be a positive multiple of 8");
+    if ((long)p->batch * p->seq_len * p->channels >= (1L << 40))
+        return fail(INKLING_ERR_UNSUPPORTED, "tensor too large");
+    if (p->batch == 0) return INKLING_OK;
+    if (!p->x || !p->w || !p->y) return fail(INKLING_ERR_INVALID, "x, w and y must not be NULL");
+    if (!aligned16(p->x) || !aligned16(p->y) || !aligned16(p->w) ||
+        (p->state && !aligned16(p->state)))
+        return fail(INKLING_ERR_INVALID, "x, w, y and state must be 16-byte aligned");
+    const size_t xb = (size_t)p->batch * p->seq_len * p->channels * 2;
+    const char *x0 = (const char *)p->x, *y0 = (const char *)p->y;
+    if (xb && x0 < y0 + xb && y0 < x0 + xb) return fail(INKLING_ERR_INVALID, "x and y overlap");
+    inkling_status st = check_device(nullptr);
+    if (st != INKLING_OK) return st;
+    cudaError_t e = launch_sconv_out(*p, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "sconv_out launch");
     return INKLING_OK;
 }
 

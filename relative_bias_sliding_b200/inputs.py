@@ -95,6 +95,21 @@ class ChunkSpec:
         return 4 * self.d * self.Hq * self.B * self.allowed_pairs
 
 
+@dataclass(frozen=True)
+class SconvOutSpec:
+    """Output sconv over the attention output [B, T, Hq*128] with a state."""
+    name: str
+    B: int
+    T: int
+    C: int
+    seed: int
+
+    @property
+    def bytes_moved(self) -> int:
+        """x read once and y written once (bf16); the state is negligible."""
+        return 2 * self.B * self.T * self.C * 2
+
+
 WORKLOADS = {
     # tiny full-causal prefill, small enough for the oracle on every row
     "prefill_tiny_b1_t256": PrefillSpec("prefill_tiny_b1_t256", 1, 256, 8, 1, 128, 0, 256,
@@ -121,6 +136,8 @@ WORKLOADS = {
     # 2048-token chunk (the sliding-window prefill's shape, cut in chunks)
     "prefill_chunked_swa_b4_c2048": ChunkSpec("prefill_chunked_swa_b4_c2048", 4, 6144, 2048, 64,
                                               8, 128, 4096, 4096, 1.0, 5),
+    # output sconv over the sliding-window prefill's attention output
+    "sconv_out_b4_t8192": SconvOutSpec("sconv_out_b4_t8192", 4, 8192, 64 * 128, 6),
     # smaller cuts of the same workloads for profiler captures (still larger
     # than L2, a few GB on the device at most)
     "prefill_swa_b1_t8192": PrefillSpec("prefill_swa_b1_t8192", 1, 8192, 64, 8, 128, 4096,
@@ -248,4 +265,12 @@ def make_chunk(spec: ChunkSpec, device="cpu"):
     return dict(q=q, cu_q=cu_q, k_new=k_new, v_new=v_new, w_k=w_k, w_v=w_v, bias=bias,
                 k_state=k_state, v_state=v_state, seq_lens=seq_lens, block_table=block_table,
                 k_cache=k_cache, v_cache=v_cache)
+
+
+def make_sconv_out(spec: SconvOutSpec, device="cpu"):
+    g = _generator(device, spec.seed)
+    x = _normal_bf16(g, (spec.B, spec.T, spec.C), device)
+    w = torch.randn((spec.C, 4), generator=g, device=device, dtype=torch.float32) * 0.5
+    state = _normal_bf16(g, (spec.B, 3, spec.C), device)
+    return dict(x=x, w=w, state=state)
 

@@ -52,6 +52,8 @@ int main(void) {{
   F(inkling_decode_params, num_splits) F(inkling_decode_params, status)
   F(inkling_decode_params, q_len) F(inkling_prefill_paged_params, cu_q)
   F(inkling_prefill_paged_params, max_q) F(inkling_prefill_paged_params, d_max)
+  printf("sconv_out %zu\\n", sizeof(inkling_sconv_out_params));
+  F(inkling_sconv_out_params, y) F(inkling_sconv_out_params, channels)
   return 0;
 }}""")
     exe = tmp_path / "sizes"
@@ -71,6 +73,10 @@ int main(void) {{
     assert int(out["inkling_prefill_paged_params cu_q"]) == P.cu_q.offset
     assert int(out["inkling_prefill_paged_params max_q"]) == P.max_q.offset
     assert int(out["inkling_prefill_paged_params d_max"]) == P.d_max.offset
+    O = binding.SconvOutParams
+    assert int(out["sconv_out"]) == ctypes.sizeof(O)
+    assert int(out["inkling_sconv_out_params y"]) == O.y.offset
+    assert int(out["inkling_sconv_out_params channels"]) == O.channels.offset
 
 
 def test_workspace_bytes(lib):
