@@ -13,6 +13,9 @@ cudaError_t launch_sconv_kv(const inkling_sconv_params &p, cudaStream_t stream);
 cudaError_t launch_attn_prefill(const inkling_prefill_params &p, const CUtensorMap *maps,
                                 cudaStream_t stream);
 cudaError_t launch_sconv_out(const inkling_sconv_out_params &p, cudaStream_t stream);
+cudaError_t launch_attn_decode_mq(const inkling_decode_params &p, int splits, void *workspace,
+                                  const CUtensorMap &tm_q, const CUtensorMap &tm_k,
+                                  const CUtensorMap &tm_v, cudaStream_t stream);
 cudaError_t launch_attn_prefill_paged(const inkling_prefill_paged_params &p, const CUtensorMap &tm_q,
                                       const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                                       cudaStream_t stream);
@@ -408,6 +411,25 @@ static inkling_status decode_with(const inkling_decode_params *p, int splits, vo
     const cuuint64_t rows = (cuuint64_t)p->num_blocks * p->num_kv_heads * 128;
     cuuint64_t dims[2] = {128, rows};
     cuuint64_t str[1] = {256};
+    if (p->q_len > 1) {
+        // multi-token decode: a whole 128-token block per key/value box, and
+        // the G x q_len query rows of a kv head in one 3-D box of
+        // q viewed as (d, head, sequence x token)
+        const int G = p->num_q_heads / p->num_kv_heads;
+        cuuint32_t box[2] = {64, 128};
+        if ((st = make_map(&tm_k, p->k_cache, 2, dims, str, box)) != INKLING_OK) return st;
+        if ((st = make_map(&tm_v, p->v_cache, 2, dims, str, box)) != INKLING_OK) return st;
+        CUtensorMap tm_q;
+        const cuuint64_t Hq = (cuuint64_t)p->num_q_heads;
+        cuuint64_t qd[3] = {128, Hq, (cuuint64_t)p->num_seqs * p->q_len};
+        cuuint64_t qs[2] = {256, Hq * 256};
+        cuuint32_t qb[3] = {64, (cuuint32_t)G, (cuuint32_t)p->q_len};
+        if ((st = make_map(&tm_q, p->q, 3, qd, qs, qb)) != INKLING_OK) return st;
+        cudaError_t e = launch_attn_decode_mq(*p, splits, workspace, tm_q, tm_k, tm_v,
+                                              (cudaStream_t)stream);
+        if (e != cudaSuccess) return cuda_fail(e, "attn_decode (multi-token) launch");
+        return INKLING_OK;
+    }
     cuuint32_t box[2] = {64, 64};
     if ((st = make_map(&tm_k, p->k_cache, 2, dims, str, box)) != INKLING_OK) return st;
     if ((st = make_map(&tm_v, p->v_cache, 2, dims, str, box)) != INKLING_OK) return st;

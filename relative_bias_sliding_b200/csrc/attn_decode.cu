@@ -41,7 +41,6 @@ struct DecodeArgs {
     float *part_ml;  // [S, Hq, splits, 2] (max in log2 units, sum)
     int32_t *status;
     int S, Hq, Hkv, G, max_blocks, num_blocks, window, d_max, splits;
-    int Q;  // query tokens per sequence (decode_mq_split_kernel)
 };
 
 INK_DEV void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
@@ -314,270 +313,6 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
     __syncthreads();
 }
 
-// Multi-token decode: Q >= 2 query tokens per sequence (the draft tokens of
-// speculative decoding / multi-token prediction; vLLM Recipes
-// "thinkingmachines/Inkling", Overview, MTP bullet: up to 9 tokens per forward
-// step).  Query qi of sequence s sits at position L - Q + qi and sees keys up
-// to itself, inside the window, with the bias at its own distance.
-//  * grid and ring as decode_split_kernel; the G*Q (token, head) rows of a
-//    kv head are cut into m-tiles of 16, one per compute warp (at most 5), and
-//    each compute warp walks every key of every 64-key chunk for its rows:
-//    S (16 x 64) = 8 k-steps x 8 n-tiles of mma.sync m16n8k16, online softmax
-//    per row, O (16 x 128) += P V with P from the S accumulators.
-//  * the last warp is the producer; no cross-warp merge (rows are disjoint);
-//    with one split the warp writes bf16 outputs, otherwise unnormalised
-//    partials for decode_combine_kernel (row index (s*Q + qi)*Hq + h).
-__global__ void __launch_bounds__(192, 1)
-decode_mq_split_kernel(const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const DecodeArgs a) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint64_t *full = (uint64_t *)(smem + kDecStages * kDecStageBytes);
-    uint64_t *empty = full + kDecStages;
-    volatile int *abort_flag = (volatile int *)(empty + kDecStages);
-
-    const int nwarps = blockDim.x >> 5, mtiles = nwarps - 1;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int s = blockIdx.x % a.S;
-    const int kvh = (blockIdx.x / a.S) % a.Hkv;
-    const int split = blockIdx.x / (a.S * a.Hkv);
-
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < kDecStages; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], mtiles);
-        }
-        *abort_flag = 0;
-        fence_mbar_init();
-    }
-    __syncthreads();
-
-    // key range of this sequence (union over its Q queries) and this split
-    const int L = a.seq_lens[s];
-    const bool bad_len = (L < a.Q || L > a.max_blocks * 128);
-    const int lo = (a.window > 0) ? max(0, L - a.Q - a.window + 1) : 0;
-    int ca = 0, cb = 0;
-    if (!bad_len) {
-        const int c_lo = lo >> 6, c_hi = (L + 63) >> 6;
-        const int per = (c_hi - c_lo + a.splits - 1) / a.splits;
-        ca = min(c_hi, c_lo + split * per);
-        cb = min(c_hi, ca + per);
-    } else if (threadIdx.x == 0 && split == 0 && kvh == 0) {
-        report_status(a.status, INKLING_STATUS_BAD_LENGTH);
-    }
-
-    if (warp == mtiles) {
-        // ------------------------------------------------------- producer --
-        int cur_batch = -1, my_id = 0, issued = 0;
-        for (int c = ca; c < cb; ++c) {
-            const int bi = c >> 1;
-            if ((bi >> 5) != cur_batch) {
-                cur_batch = bi >> 5;
-                const int idx = cur_batch * 32 + lane;
-                my_id = (idx < a.max_blocks) ? a.block_table[(long)s * a.max_blocks + idx] : 0;
-            }
-            int blk = __shfl_sync(0xffffffffu, my_id, bi & 31);
-            int ok = 1;
-            if (lane == 0) {
-                const int k = c - ca, st = k % kDecStages;
-                ok = mbar_wait(&empty[st], ((k / kDecStages) & 1) ^ 1, abort_flag, a.status);
-                if (ok) {
-                    if (blk < 0 || blk >= a.num_blocks) {
-                        report_status(a.status, INKLING_STATUS_BAD_BLOCK);
-                        blk = 0;  // keep the pipeline running on a valid block
-                    }
-                    const int row = (blk * a.Hkv + kvh) * 128 + (c & 1) * 64;
-                    uint8_t *kb = smem + st * kDecStageBytes;
-                    mbar_arrive_expect_tx(&full[st], kDecStageBytes);
-                    tma_load_2d(kb, &tm_k, &full[st], 0, row);
-                    tma_load_2d(kb + 8192, &tm_k, &full[st], 64, row);
-                    tma_load_2d(kb + 16384, &tm_v, &full[st], 0, row);
-                    tma_load_2d(kb + 24576, &tm_v, &full[st], 64, row);
-                    ++issued;
-                }
-            }
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) break;
-        }
-        if (lane == 0) {
-            for (int k = max(0, issued - kDecStages); k < issued; ++k)
-                mbar_wait(&full[k % kDecStages], (k / kDecStages) & 1, nullptr, a.status);
-        }
-    } else {
-        // --------------------------------------------------------- compute --
-        // this thread's rows: R0 = 16*warp + lane/4 and R1 = R0 + 8 of the
-        // G*Q (token, head) rows, row R = qi*G + g
-        const int g4 = lane >> 2, t = lane & 3;
-        const int rows = a.G * a.Q;
-        int qi[2], hh[2], ipos[2];
-        bool rv[2];
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            const int R = 16 * warp + g4 + 8 * r;
-            rv[r] = R < rows;
-            const int Rc = rv[r] ? R : 0;
-            qi[r] = Rc / a.G;
-            hh[r] = kvh * a.G + Rc % a.G;
-            ipos[r] = L - a.Q + qi[r];
-        }
-        uint32_t qa[8][4];
-        {
-            const uint16_t *q0 = a.q + (((long)s * a.Q + qi[0]) * a.Hq + hh[0]) * 128;
-            const uint16_t *q1 = a.q + (((long)s * a.Q + qi[1]) * a.Hq + hh[1]) * 128;
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                qa[ks][0] = rv[0] ? *(const uint32_t *)(q0 + 16 * ks + 2 * t) : 0u;
-                qa[ks][1] = rv[1] ? *(const uint32_t *)(q1 + 16 * ks + 2 * t) : 0u;
-                qa[ks][2] = rv[0] ? *(const uint32_t *)(q0 + 16 * ks + 8 + 2 * t) : 0u;
-                qa[ks][3] = rv[1] ? *(const uint32_t *)(q1 + 16 * ks + 8 + 2 * t) : 0u;
-            }
-        }
-        const float kLog2e = 1.4426950408889634f;
-        const float c1 = kLog2e * 0.08838834764831845f;  // log2(e) / sqrt(128)
-        const float *bias0 = a.bias + (long)hh[0] * (a.d_max + 1);
-        const float *bias1 = a.bias + (long)hh[1] * (a.d_max + 1);
-
-        float o[16][4];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-        float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
-
-        const uint32_t sbase = smem_u32(smem);
-        for (int c = ca; c < cb; ++c) {
-            const int k = c - ca, st = k % kDecStages;
-            // bias of this thread's 16 keys for both rows, fetched before the
-            // wait (0 for keys the row may not see)
-            float bv[8][4];
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int r = e >> 1;
-                    const int j = c * 64 + nt * 8 + 2 * t + (e & 1);
-                    const int dist = ipos[r] - j;
-                    const bool ok = rv[r] && dist >= 0 && (a.window <= 0 || dist < a.window);
-                    bv[nt][e] = ok ? __ldg((r ? bias1 : bias0) + min(dist, a.d_max)) : 0.f;
-                }
-            if (!mbar_wait_warp(&full[st], (k / kDecStages) & 1, abort_flag, a.status)) break;
-
-            const uint32_t kst = sbase + st * kDecStageBytes;
-            const uint32_t vst = kst + 16384;
-            // S = Q K^T: 16 rows x 64 keys
-            float sacc[8][4];
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                const int r = 16 * p + ((lane >> 4) & 1) * 8 + (lane & 7);
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const int cc = 2 * (ks & 3) + ((lane >> 3) & 1);
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4(kst + (ks >> 2) * 8192 + sw128_off(r, cc), b0, b1, b2, b3);
-                    mma16816(sacc[2 * p], qa[ks], b0, b1);
-                    mma16816(sacc[2 * p + 1], qa[ks], b2, b3);
-                }
-            }
-            // logits (log2 units), mask, online softmax per row
-            float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int r = e >> 1;
-                    const int j = c * 64 + nt * 8 + 2 * t + (e & 1);
-                    const int dist = ipos[r] - j;
-                    const bool ok = rv[r] && dist >= 0 && (a.window <= 0 || dist < a.window);
-                    sacc[nt][e] = ok ? fmaf(sacc[nt][e], c1, bv[nt][e] * kLog2e) : -INFINITY;
-                    mx[r] = fmaxf(mx[r], sacc[nt][e]);
-                }
-            float alpha[2];
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
-                mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
-                const float m_new = fmaxf(m[r], mx[r]);
-                alpha[r] = (m[r] == -INFINITY) ? 0.f : ex2(m[r] - m_new);
-                m[r] = m_new;
-            }
-            float psum[2] = {0.f, 0.f};
-            uint32_t pa[4][4];
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt) {
-                float p4[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int r = e >> 1;
-                    p4[e] = (sacc[nt][e] == -INFINITY) ? 0.f : ex2(sacc[nt][e] - m[r]);
-                    psum[r] += p4[e];
-                }
-                // A fragment of k-step nt/2: rows g4 / g4+8, keys 2t, 2t+1 (+8)
-                pa[nt >> 1][(nt & 1) * 2 + 0] = pack_bf16(p4[0], p4[1]);
-                pa[nt >> 1][(nt & 1) * 2 + 1] = pack_bf16(p4[2], p4[3]);
-            }
-#pragma unroll
-            for (int r = 0; r < 2; ++r) l[r] = l[r] * alpha[r] + psum[r];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                o[i][0] *= alpha[0];
-                o[i][1] *= alpha[0];
-                o[i][2] *= alpha[1];
-                o[i][3] *= alpha[1];
-            }
-            // O += P V: 4 k-steps of 16 keys, 16 n-tiles of 8 head-dim columns
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint32_t af[4] = {pa[kk][0], pa[kk][1], pa[kk][2], pa[kk][3]};
-                const int r = 16 * kk + ((lane >> 3) & 1) * 8 + (lane & 7);
-#pragma unroll
-                for (int mm = 0; mm < 8; ++mm) {
-                    const int ch = 2 * mm + (lane >> 4);  // 16-byte chunk of d
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4_t(vst + (ch >> 3) * 8192 + sw128_off(r, ch & 7), b0, b1, b2, b3);
-                    mma16816(o[2 * mm], af, b0, b1);
-                    mma16816(o[2 * mm + 1], af, b2, b3);
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[st]);
-        }
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            l[r] += __shfl_xor_sync(0xffffffffu, l[r], 1);
-            l[r] += __shfl_xor_sync(0xffffffffu, l[r], 2);
-        }
-        if (!*abort_flag && !bad_len) {
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                if (!rv[r]) continue;
-                const long pair = ((long)s * a.Q + qi[r]) * a.Hq + hh[r];
-                if (a.splits == 1) {
-                    const float inv = (l[r] > 0.f) ? 1.f / l[r] : 0.f;
-                    uint16_t *orow = a.out + pair * 128;
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        *(uint32_t *)(orow + i * 8 + 2 * t) =
-                            pack_bf16(o[i][2 * r] * inv, o[i][2 * r + 1] * inv);
-                    if (a.lse && t == 0)
-                        a.lse[pair] =
-                            (l[r] > 0.f) ? (m[r] + __log2f(l[r])) * 0.6931471805599453f : -INFINITY;
-                } else {
-                    const long pi = pair * a.splits + split;
-                    float *po = a.part_o + pi * 128;
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        *(float2 *)(po + i * 8 + 2 * t) = make_float2(o[i][2 * r], o[i][2 * r + 1]);
-                    if (t == 0) {
-                        a.part_ml[pi * 2] = m[r];
-                        a.part_ml[pi * 2 + 1] = l[r];
-                    }
-                }
-            }
-        }
-    }
-    __syncthreads();
-}
-
 // One warp per (sequence, query head): log-sum-exp merge of the splits.
 __global__ void __launch_bounds__(128)
 decode_combine_kernel(const float *__restrict__ part_o, const float *__restrict__ part_ml,
@@ -613,6 +348,13 @@ decode_combine_kernel(const float *__restrict__ part_o, const float *__restrict_
         lse[pair] = (Ls > 0.f) ? (M + __log2f(Ls)) * 0.6931471805599453f : -INFINITY;
 }
 
+cudaError_t launch_decode_combine(const float *part_o, const float *part_ml, uint16_t *out, float *lse,
+                                  long rows, int splits, cudaStream_t stream) {
+    decode_combine_kernel<<<(unsigned)((rows + 3) / 4), 128, 0, stream>>>(part_o, part_ml, out, lse,
+                                                                        (int)rows, splits);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_attn_decode(const inkling_decode_params &p, int splits, void *workspace,
                                const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                                cudaStream_t stream) {
@@ -635,23 +377,13 @@ cudaError_t launch_attn_decode(const inkling_decode_params &p, int splits, void 
     a.window = p.window;
     a.d_max = p.d_max;
     a.splits = splits;
-    a.Q = p.q_len > 1 ? p.q_len : 1;
-    const long rows_total = pairs * a.Q;  // (sequence, token, head) rows
+    const long rows_total = pairs;
     a.part_ml = splits > 1 ? (float *)workspace + rows_total * splits * 128 : nullptr;
     const long grid = (long)p.num_seqs * p.num_kv_heads * splits;
-    if (a.Q == 1) {
-        cudaError_t e0 = cudaFuncSetAttribute(decode_split_kernel,
-                                              cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
-        if (e0 != cudaSuccess) return e0;
-        decode_split_kernel<<<(unsigned)grid, 160, kDecSmem, stream>>>(tm_k, tm_v, a);
-    } else {
-        cudaError_t e0 = cudaFuncSetAttribute(decode_mq_split_kernel,
-                                              cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
-        if (e0 != cudaSuccess) return e0;
-        const int mtiles = (a.G * a.Q + 15) / 16;  // 1..5 (checked by the caller)
-        decode_mq_split_kernel<<<(unsigned)grid, 32 * (mtiles + 1), kDecSmem, stream>>>(tm_k, tm_v,
-                                                                                          a);
-    }
+    cudaError_t e0 = cudaFuncSetAttribute(decode_split_kernel,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
+    if (e0 != cudaSuccess) return e0;
+    decode_split_kernel<<<(unsigned)grid, 160, kDecSmem, stream>>>(tm_k, tm_v, a);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || splits == 1) return e;
     decode_combine_kernel<<<(unsigned)((rows_total + 3) / 4), 128, 0, stream>>>(

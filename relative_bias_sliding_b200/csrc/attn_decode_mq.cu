@@ -1,0 +1,453 @@
+// attn_decode_mq.cu — multi-token decode on tcgen05 tensor cores: the q_len
+// newest tokens of each sequence (the draft tokens of speculative decoding /
+// multi-token prediction; vLLM Recipes "thinkingmachines/Inkling", Overview,
+// MTP bullet: up to 9 tokens per forward step) attend to the paged cache.
+// Query qi of sequence s sits at position L - q_len + qi and sees keys up to
+// itself, inside the window, with the bias at its own distance.
+//
+// One thread block = one (sequence, kv head, split).  All G * q_len (token,
+// head) rows of the kv head (at most 80) form one 128-row tile: a single 3-D
+// TMA box gathers them (q viewed as [S*q_len, Hq, d], box {64, G, q_len}),
+// rows ordered r = qi*G + g.  Each 128-token cache block is one key tile
+// (two 64-column TMA boxes each for keys and values, 128-byte swizzle).
+//   S = Q K^T: tcgen05 M=128 N=128 into one of two TMEM buffers, so the MMA
+//     of key tile k+1 runs while the softmax works on tile k;
+//   P (bf16) over the first 64 columns of its S buffer; O += P V (TMEM A);
+//   the softmax (4 warps, thread = row = TMEM lane) reads each row's bias
+//     from per-head diagonals staged in shared memory (4 shifted copies, so a
+//     row's 128 values come in 32 aligned 16-byte loads), masks the row's
+//     columns outside its causal/window range, and rescales O only when its
+//     running maximum grows by more than 8 (log2 units), after the previous
+//     P.V has completed.
+// The key range of a sequence (union of its rows' windows) is cut into
+// `splits` runs of tiles on separate blocks; with more than one split the
+// block writes unnormalised partials (max in log2 units, sum, O) that
+// decode_combine_kernel merges, as for single-token decode.
+#include "common.cuh"
+
+#include <type_traits>
+
+namespace inkling {
+
+cudaError_t launch_decode_combine(const float *part_o, const float *part_ml, uint16_t *out, float *lse,
+                                  long rows, int splits, cudaStream_t stream);
+
+constexpr int kMqCopy = 148;                      // floats per shifted copy (>= 127 + 10 + 3)
+constexpr int kMqHead = 4 * kMqCopy + 20;         // floats per head (== 4 mod 32: the 8 heads
+                                                  // of a quarter warp hit distinct banks)
+constexpr int kMqBiasBuf = 8 * kMqHead;           // 8 heads x 4 copies
+constexpr uint32_t MQ_Q = 0;                      // 128 rows x 256 B (two 16 KB halves)
+constexpr uint32_t MQ_K = 32768;                  // 2 stages x 32 KB
+constexpr uint32_t MQ_V = 98304;                  // 2 stages x 32 KB
+constexpr uint32_t MQ_BIAS = 163840;              // 2 buffers of staged diagonals
+constexpr uint32_t MQ_BAR = MQ_BIAS + 2 * kMqBiasBuf * 4;
+constexpr int kMqSmem = MQ_BAR + 256 + 1024;
+
+enum {
+    M_QFULL = 0,
+    M_KFULL = 1,    // +stage
+    M_VFULL = 3,
+    M_KEMPTY = 5,
+    M_VEMPTY = 7,
+    M_SFULL = 9,    // +S buffer
+    M_PFULL = 11,   // +S buffer (128 arrivals)
+    M_OREADY = 13,  // one phase per P.V issued
+    M_DRAIN = 14,
+    M_COUNT = 15
+};
+
+struct DecodeMqArgs {
+    const int32_t *block_table, *seq_lens;
+    const float *bias;
+    uint16_t *out;
+    float *lse;
+    float *part_o, *part_ml;
+    int32_t *status;
+    int S, Q, Hq, Hkv, G, max_blocks, num_blocks, window, d_max, splits;
+};
+
+__global__ void __launch_bounds__(192, 1)
+decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const DecodeMqArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const uint32_t sb = smem_u32(smem);
+    uint64_t *bar = (uint64_t *)(smem + MQ_BAR);
+    uint32_t *tmem_slot = (uint32_t *)(bar + M_COUNT);
+    volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int s = blockIdx.x % a.S;
+    const int kvh = (blockIdx.x / a.S) % a.Hkv;
+    const int split = blockIdx.x / (a.S * a.Hkv);
+    const int Q = a.Q, G = a.G, rows = G * Q;
+
+    // key tiles of this sequence (union of its rows' windows) and this split
+    const int L = a.seq_lens[s];
+    const bool bad_len = (L < Q || L > a.max_blocks * 128);
+    const int klo = (a.window > 0) ? max(0, L - Q - a.window + 1) : 0;
+    int ta = 0, tb = 0;
+    if (!bad_len) {
+        const int t_lo = klo >> 7, t_hi = (L - 1) >> 7;
+        const int per = (t_hi - t_lo + a.splits) / a.splits;
+        ta = min(t_hi + 1, t_lo + split * per);
+        tb = min(t_hi + 1, ta + per);
+    } else if (threadIdx.x == 0 && split == 0 && kvh == 0) {
+        report_status(a.status, INKLING_STATUS_BAD_LENGTH);
+    }
+    const int nt = tb - ta;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < M_COUNT; ++i)
+            mbar_init(&bar[i], (i == M_PFULL || i == M_PFULL + 1) ? 128 : 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+
+    if (warp < 4) {
+        // ============================================ softmax (thread = row) ==
+        const int u = threadIdx.x;
+        const bool rv = u < rows;
+        // a warp whose 32 rows are all padding (G * q_len <= 96) computes
+        // nothing: it stages bias, keeps the barrier and arrives on P_FULL
+        // (its P rows are never read for an output)
+        const bool live = warp * 32 < rows;
+        const int qi = rv ? u / G : 0, g = rv ? u % G : 0;
+        const int h = kvh * G + g;
+        const int ipos = L - Q + qi;  // this row's query position
+        const uint32_t tl = tbase + ((uint32_t)(warp * 32) << 16);
+        const uint32_t o_col = tl + 256;
+        const float scale = 0.08838834764831845f;  // 1/sqrt(128)
+        const float kLog2e = 1.4426950408889634f;
+        const float kTau = 5.545177444479562f;     // 8 ln 2
+        const int W = a.window, Dm = a.d_max;
+        float m_ref = -INFINITY, l = 0.f;
+        const int o_rd = Q - 1 - qi, sh = o_rd & 3;  // start of this row in its head's diagonal
+        const int span = Q + 127 + 3;                // staged values per head
+        bool dead = bad_len;
+        // diagonal of head g for key tile k: R[kk] = bias[h_g, clamp(L-1-j0-kk, 0, d_max)]
+        // (row qi reads R[Q-1-qi + c] for column c), as 4 copies shifted by
+        // 0..3 floats; thread t holds elements t, t+128, ... of the G x span
+        // values, fetched one tile ahead and stored under the next barrier
+        constexpr int kPer = (8 * (10 + 130) + 127) / 128;  // values per thread, G <= 8, Q <= 10
+        float nxt[kPer];
+        // this thread's (head, offset) pairs, the same for every tile (-1: none)
+        int egg[kPer], ekk[kPer];
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const int e = threadIdx.x + 128 * i;
+            egg[i] = e < G * span ? e / span : -1;
+            ekk[i] = e < G * span ? e % span : 0;
+        }
+        auto fetch = [&](int k) {
+            const int top = L - 1 - (ta + k) * 128;
+#pragma unroll
+            for (int i = 0; i < kPer; ++i)
+                if (egg[i] >= 0)
+                    nxt[i] = __ldg(a.bias + (long)(kvh * G + egg[i]) * (Dm + 1) +
+                                   min(max(top - ekk[i], 0), Dm));
+        };
+        auto stage = [&](int k) {
+            float *bb = (float *)(smem + MQ_BIAS) + (k & 1) * kMqBiasBuf;
+#pragma unroll
+            for (int i = 0; i < kPer; ++i) {
+                if (egg[i] < 0) continue;
+#pragma unroll
+                for (int s4 = 0; s4 < 4; ++s4)
+                    if (ekk[i] >= s4) bb[egg[i] * kMqHead + s4 * kMqCopy + ekk[i] - s4] = nxt[i];
+            }
+        };
+        if (nt > 0) {
+            fetch(0);
+            stage(0);
+        }
+        for (int k = 0; k < nt; ++k) {
+            const int j0 = (ta + k) * 128;
+            float *bb = (float *)(smem + MQ_BIAS) + (k & 1) * kMqBiasBuf;
+            named_bar_sync(1, 128);  // tile k's diagonals are staged; tile k-1's reads are done
+            if (k + 1 < nt) fetch(k + 1);
+            if (!live) {
+                mbar_arrive(&bar[M_PFULL + (k & 1)]);
+                if (k + 1 < nt) stage(k + 1);
+                continue;
+            }
+            if (!dead) dead = !mbar_wait_warp(&bar[M_SFULL + (k & 1)], (k >> 1) & 1, abort_flag, a.status);
+            if (dead) {
+                if (k + 1 < nt) stage(k + 1);
+                continue;  // keep stepping through the group barrier
+            }
+            tc_fence_after();
+            const uint32_t s_col = tl + (k & 1) * 128;
+            uint32_t sr[128];
+            tmem_ld32(s_col + 0, sr + 0);
+            tmem_ld32(s_col + 32, sr + 32);
+            tmem_ld32(s_col + 64, sr + 64);
+            tmem_ld32(s_col + 96, sr + 96);
+            tmem_wait_ld();
+            // columns this row may see: ipos - j0 - c in [0, W)
+            const int dist0 = ipos - j0;
+            const int cmax = rv ? min(127, dist0) : -1;
+            const int cmin = (W > 0) ? max(0, dist0 - W + 1) : 0;
+            const bool full = cmin == 0 && cmax == 127;
+            const float4 *rp = (const float4 *)(bb + g * kMqHead + sh * kMqCopy + (o_rd - sh));
+            float x[128];
+            float m8[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
+            const f32x2 sc2 = pk2(scale, scale);
+            auto logits = [&](auto masked) {
+#pragma unroll
+                for (int cb = 0; cb < 4; ++cb) {
+                    float4 b4[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) b4[j] = rp[cb * 8 + j];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int c = 32 * cb + 4 * j;
+                        const f32x2 xa = ffma2(pk2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])),
+                                               sc2, pk2(b4[j].x, b4[j].y));
+                        const f32x2 xb = ffma2(pk2(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3])),
+                                               sc2, pk2(b4[j].z, b4[j].w));
+                        upk2(xa, x[c], x[c + 1]);
+                        upk2(xb, x[c + 2], x[c + 3]);
+                        if (decltype(masked)::value) {
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                x[c + e] = (c + e >= cmin && c + e <= cmax) ? x[c + e] : -INFINITY;
+                        }
+                        m8[j] = max3f(max3f(m8[j], x[c], x[c + 1]), x[c + 2], x[c + 3]);
+                    }
+                }
+            };
+            if (full)
+                logits(std::false_type{});
+            else
+                logits(std::true_type{});
+            const float mx =
+                fmaxf(max3f(m8[0], m8[1], m8[2]), max3f(max3f(m8[3], m8[4], m8[5]), m8[6], m8[7]));
+            const bool grow = mx > m_ref + kTau;
+            float alpha = 1.f;
+            if (grow) {
+                alpha = ex2((m_ref - mx) * kLog2e);
+                l *= alpha;
+                m_ref = mx;
+            }
+            const float mneg = (m_ref == -INFINITY) ? 0.f : -m_ref * kLog2e;
+            {
+                const f32x2 l2e2 = pk2(kLog2e, kLog2e), mneg2 = pk2(mneg, mneg);
+                f32x2 acc[4] = {0ull, 0ull, 0ull, 0ull};
+                uint32_t pk[64];
+#pragma unroll
+                for (int c = 0; c < 64; ++c) {
+                    const f32x2 tt = ffma2(pk2(x[2 * c], x[2 * c + 1]), l2e2, mneg2);
+                    float t0, t1;
+                    upk2(tt, t0, t1);
+                    const float p0 = ex2(t0), p1 = ex2(t1);
+                    acc[c & 3] = fadd2(acc[c & 3], pk2(p0, p1));
+                    pk[c] = pack_bf16(p0, p1);
+                }
+                tmem_st32(s_col + 0, pk + 0);
+                tmem_st32(s_col + 32, pk + 32);
+                const f32x2 s01 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+                float la, lb;
+                upk2(s01, la, lb);
+                l += la + lb;
+            }
+            // O rescale, after the previous tile's P.V has completed (at most
+            // that phase can have completed: the next P.V waits for this P)
+            if (k > 0 && __any_sync(0xffffffffu, grow)) {
+                if (!mbar_wait_warp(&bar[M_OREADY], (k - 1) & 1, abort_flag, a.status)) {
+                    dead = true;
+                } else {
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int cb = 0; cb < 4; ++cb) {
+                        uint32_t orr[32];
+                        tmem_ld32(o_col + cb * 32, orr);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
+                        tmem_st32(o_col + cb * 32, orr);
+                    }
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bar[M_PFULL + (k & 1)]);
+            if (k + 1 < nt) stage(k + 1);
+        }
+        // epilogue: the last P.V has completed
+        const bool have_o = live && !dead && nt > 0 &&
+                            mbar_wait_warp(&bar[M_OREADY], (nt - 1) & 1, abort_flag, a.status);
+        if (have_o) tc_fence_after();
+        uint32_t ob[128];
+        if (have_o) {
+#pragma unroll
+            for (int cb = 0; cb < 4; ++cb) tmem_ld32(o_col + cb * 32, ob + cb * 32);
+            tmem_wait_ld();
+        }
+        auto o = [&](int i) { return __uint_as_float(ob[i]); };
+        if (rv && !bad_len && !*abort_flag) {
+            const long pair = ((long)s * Q + qi) * a.Hq + h;
+            if (a.splits == 1) {
+                const float inv = (l > 0.f) ? 1.f / l : 0.f;
+                uint4 *dst = (uint4 *)(a.out + pair * 128);
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    uint4 v;
+                    v.x = pack_bf16(o(8 * c + 0) * inv, o(8 * c + 1) * inv);
+                    v.y = pack_bf16(o(8 * c + 2) * inv, o(8 * c + 3) * inv);
+                    v.z = pack_bf16(o(8 * c + 4) * inv, o(8 * c + 5) * inv);
+                    v.w = pack_bf16(o(8 * c + 6) * inv, o(8 * c + 7) * inv);
+                    dst[c] = v;
+                }
+                if (a.lse) a.lse[pair] = (l > 0.f) ? m_ref + __logf(l) : -INFINITY;
+            } else {
+                const long pi = pair * a.splits + split;
+                float4 *po = (float4 *)(a.part_o + pi * 128);
+                if (have_o) {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        po[c] = make_float4(o(4 * c), o(4 * c + 1), o(4 * c + 2), o(4 * c + 3));
+                }
+                // an empty split (or row) contributes nothing: max -inf
+                a.part_ml[pi * 2] = (have_o && l > 0.f) ? m_ref * kLog2e : -INFINITY;
+                a.part_ml[pi * 2 + 1] = have_o ? l : 0.f;
+            }
+        }
+    } else if (warp == 4 && lane == 0) {
+        // ============================================== TMA producer ==
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        if (nt > 0) {
+            mbar_arrive_expect_tx(&bar[M_QFULL], 2 * rows * 128);
+            tma_load_3d(smem + MQ_Q, &tm_q, &bar[M_QFULL], 0, kvh * G, s * Q);
+            tma_load_3d(smem + MQ_Q + 16384, &tm_q, &bar[M_QFULL], 64, kvh * G, s * Q);
+        }
+        int issued = 0;
+        for (int k = 0; k < nt; ++k) {
+            const int st = k & 1;
+            const uint32_t ph = ((k >> 1) & 1) ^ 1;
+            int blk = a.block_table[(long)s * a.max_blocks + ta + k];
+            if (blk < 0 || blk >= a.num_blocks) {
+                report_status(a.status, INKLING_STATUS_BAD_BLOCK);
+                blk = 0;  // keep the pipeline running on a valid block
+            }
+            const int row = (blk * a.Hkv + kvh) * 128;
+            if (!mbar_wait(&bar[M_KEMPTY + st], ph, abort_flag, a.status)) break;
+            mbar_arrive_expect_tx(&bar[M_KFULL + st], 32768);
+            tma_load_2d(smem + MQ_K + st * 32768, &tm_k, &bar[M_KFULL + st], 0, row);
+            tma_load_2d(smem + MQ_K + st * 32768 + 16384, &tm_k, &bar[M_KFULL + st], 64, row);
+            if (!mbar_wait(&bar[M_VEMPTY + st], ph, abort_flag, a.status)) break;
+            mbar_arrive_expect_tx(&bar[M_VFULL + st], 32768);
+            tma_load_2d(smem + MQ_V + st * 32768, &tm_v, &bar[M_VFULL + st], 0, row);
+            tma_load_2d(smem + MQ_V + st * 32768 + 16384, &tm_v, &bar[M_VFULL + st], 64, row);
+            ++issued;
+        }
+        // drain: every load issued has landed before the block may exit
+        if (nt > 0) mbar_wait(&bar[M_QFULL], 0, nullptr, a.status);
+        for (int k = max(0, issued - 2); k < issued; ++k) {
+            mbar_wait(&bar[M_KFULL + (k & 1)], (k >> 1) & 1, nullptr, a.status);
+            mbar_wait(&bar[M_VFULL + (k & 1)], (k >> 1) & 1, nullptr, a.status);
+        }
+    } else if (warp == 5 && lane == 0) {
+        // ================================================ MMA issuer ==
+        const uint32_t id_qk = idesc_bf16(128, 128, 0, 0);
+        const uint32_t id_pv = idesc_bf16(128, 128, 0, 1);
+        auto issue_qk = [&](int k) {
+            const int st = k & 1;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
+                const uint64_t ad = sw128_desc(sb + MQ_Q + koff, 16, 1024);
+                const uint64_t bd = sw128_desc(sb + MQ_K + st * 32768 + koff, 16, 1024);
+                umma_ss(tbase + (k & 1) * 128, ad, bd, id_qk, ks > 0 ? 1u : 0u);
+            }
+        };
+        auto issue_pv = [&](int k) {
+            const int st = k & 1;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint64_t bd = sw128_desc(sb + MQ_V + st * 32768 + ks * 2048, 16384, 1024);
+                umma_ts(tbase + 256, tbase + (k & 1) * 128 + ks * 8, bd, id_pv,
+                        (k > 0 || ks > 0) ? 1u : 0u);
+            }
+        };
+        bool alive = nt == 0 || mbar_wait(&bar[M_QFULL], 0, abort_flag, a.status);
+        // QK(0) QK(1) | PV(0) QK(2) | PV(1) QK(3) | ...: the QK^T of the next
+        // tile runs while the softmax works on the current one
+        for (int k = 0; k <= nt && alive; ++k) {
+            if (k < nt) {
+                if (!mbar_wait(&bar[M_KFULL + (k & 1)], (k >> 1) & 1, abort_flag, a.status)) break;
+                tc_fence_after();
+                issue_qk(k);
+                tc_commit(&bar[M_SFULL + (k & 1)]);
+                tc_commit(&bar[M_KEMPTY + (k & 1)]);
+            }
+            if (k >= 1) {
+                const int kp = k - 1;
+                if (!mbar_wait(&bar[M_PFULL + (kp & 1)], (kp >> 1) & 1, abort_flag, a.status) ||
+                    !mbar_wait(&bar[M_VFULL + (kp & 1)], (kp >> 1) & 1, abort_flag, a.status))
+                    break;
+                tc_fence_after();
+                issue_pv(kp);
+                tc_commit(&bar[M_OREADY]);
+                tc_commit(&bar[M_VEMPTY + (kp & 1)]);
+            }
+        }
+        // every MMA issued has completed before TMEM is released
+        tc_commit(&bar[M_DRAIN]);
+        mbar_wait(&bar[M_DRAIN], 0, nullptr, a.status);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tbase, 512);
+    }
+}
+
+cudaError_t launch_attn_decode_mq(const inkling_decode_params &p, int splits, void *workspace,
+                                  const CUtensorMap &tm_q, const CUtensorMap &tm_k,
+                                  const CUtensorMap &tm_v, cudaStream_t stream) {
+    DecodeMqArgs a;
+    a.block_table = p.block_table;
+    a.seq_lens = p.seq_lens;
+    a.bias = p.bias;
+    a.out = (uint16_t *)p.out;
+    a.lse = p.lse;
+    a.status = p.status;
+    a.S = p.num_seqs;
+    a.Q = p.q_len;
+    a.Hq = p.num_q_heads;
+    a.Hkv = p.num_kv_heads;
+    a.G = p.num_q_heads / p.num_kv_heads;
+    a.max_blocks = p.max_blocks;
+    a.num_blocks = p.num_blocks;
+    a.window = p.window;
+    a.d_max = p.d_max;
+    a.splits = splits;
+    const long rows_total = (long)p.num_seqs * p.q_len * p.num_q_heads;
+    a.part_o = (float *)workspace;
+    a.part_ml = splits > 1 ? (float *)workspace + rows_total * splits * 128 : nullptr;
+    cudaError_t e = cudaFuncSetAttribute(decode_mq_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kMqSmem);
+    if (e != cudaSuccess) return e;
+    const long grid = (long)p.num_seqs * p.num_kv_heads * splits;
+    decode_mq_tc_kernel<<<(unsigned)grid, 192, kMqSmem, stream>>>(tm_q, tm_k, tm_v, a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || splits == 1) return e;
+    return launch_decode_combine(a.part_o, a.part_ml, a.out, a.lse, rows_total, splits, stream);
+}
+
+}  // namespace inkling

@@ -6,8 +6,9 @@
 // t = 0 taken from a rolling state (or zero), one bf16 rounding.
 //
 // One thread owns 8 consecutive channels of one sequence and a run of up to
-// kOutRun consecutive tokens: history from the state (first run) or from x,
-// 16-byte loads and stores, the same fp32 FMA order as the key/value sconv.
+// kOutRun (64) consecutive tokens, with 4 row loads in flight: history from the
+// state (first run) or from x, 16-byte loads and stores, the same fp32 FMA
+// order as the key/value sconv.
 // The first run's thread also writes the new state (the last 3 raw rows of
 // (old state, x)) after reading the old one.  HBM-bound: x read once (plus 3
 // history rows per run), y written once.
@@ -15,7 +16,7 @@
 
 namespace inkling {
 
-constexpr int kOutRun = 32;
+constexpr int kOutRun = 64;
 
 __global__ void __launch_bounds__(128)
 sconv_out_kernel(const uint4 *__restrict__ x, const float4 *__restrict__ w, uint4 *state,
@@ -51,6 +52,7 @@ sconv_out_kernel(const uint4 *__restrict__ x, const float4 *__restrict__ w, uint
     unpack8(r3, h3);
     unpack8(r2, h2);
     unpack8(r1, h1);
+#pragma unroll 4
     for (int t = t0; t < t1; ++t) {
         float xv[8];
         unpack8(row(t), xv);
