@@ -412,11 +412,11 @@ static inkling_status decode_with(const inkling_decode_params *p, int splits, vo
     cuuint64_t dims[2] = {128, rows};
     cuuint64_t str[1] = {256};
     if (p->q_len > 1) {
-        // multi-token decode: a whole 128-token block per key/value box, and
+        // multi-token decode: half a block (64 tokens) per key/value box, and
         // the G x q_len query rows of a kv head in one 3-D box of
         // q viewed as (d, head, sequence x token)
         const int G = p->num_q_heads / p->num_kv_heads;
-        cuuint32_t box[2] = {64, 128};
+        cuuint32_t box[2] = {64, 64};
         if ((st = make_map(&tm_k, p->k_cache, 2, dims, str, box)) != INKLING_OK) return st;
         if ((st = make_map(&tm_v, p->v_cache, 2, dims, str, box)) != INKLING_OK) return st;
         CUtensorMap tm_q;

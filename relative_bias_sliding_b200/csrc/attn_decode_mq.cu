@@ -8,17 +8,19 @@
 // One thread block = one (sequence, kv head, split).  All G * q_len (token,
 // head) rows of the kv head (at most 80) form one 128-row tile: a single 3-D
 // TMA box gathers them (q viewed as [S*q_len, Hq, d], box {64, G, q_len}),
-// rows ordered r = qi*G + g.  Each 128-token cache block is one key tile
-// (two 64-column TMA boxes each for keys and values, 128-byte swizzle).
-//   S = Q K^T: tcgen05 M=128 N=128 into one of two TMEM buffers, so the MMA
+// rows ordered r = qi*G + g.  Key tiles are 64 tokens, half a cache block
+// (two 64-column TMA boxes each for keys and values, 128-byte swizzle), so a
+// block needs ~105 KB of shared memory and 256 TMEM columns and two blocks
+// share an SM: one's softmax runs while the other waits on its tiles.
+//   S = Q K^T: tcgen05 M=128 N=64 into one of two TMEM buffers, so the MMA
 //     of key tile k+1 runs while the softmax works on tile k;
-//   P (bf16) over the first 64 columns of its S buffer; O += P V (TMEM A);
+//   P (bf16) over the first 32 columns of its S buffer; O += P V (TMEM A);
 //   the softmax (4 warps, thread = row = TMEM lane) reads each row's bias
-//     from per-head diagonals staged in shared memory (4 shifted copies, so a
-//     row's 128 values come in 32 aligned 16-byte loads), masks the row's
-//     columns outside its causal/window range, and rescales O only when its
-//     running maximum grows by more than 8 (log2 units), after the previous
-//     P.V has completed.
+//     from per-head diagonals staged in shared memory (head stride 4 mod 32
+//     floats: the 4 tokens x 8 heads of a warp hit distinct banks), masks the
+//     row's columns outside its causal/window range, and rescales O only when
+//     its running maximum grows by more than 8 (log2 units), after the
+//     previous P.V has completed.
 // The key range of a sequence (union of its rows' windows) is cut into
 // `splits` runs of tiles on separate blocks; with more than one split the
 // block writes unnormalised partials (max in log2 units, sum, O) that
@@ -32,14 +34,13 @@ namespace inkling {
 cudaError_t launch_decode_combine(const float *part_o, const float *part_ml, uint16_t *out, float *lse,
                                   long rows, int splits, cudaStream_t stream);
 
-constexpr int kMqCopy = 148;                      // floats per shifted copy (>= 127 + 10 + 3)
-constexpr int kMqHead = 4 * kMqCopy + 20;         // floats per head (== 4 mod 32: the 8 heads
-                                                  // of a quarter warp hit distinct banks)
-constexpr int kMqBiasBuf = 8 * kMqHead;           // 8 heads x 4 copies
+constexpr int kMqTile = 64;                       // keys per tile (half a cache block)
+constexpr int kMqHead = 100;                      // floats per head diagonal (>= 63 + 10, == 4 mod 32)
+constexpr int kMqBiasBuf = 8 * kMqHead;
 constexpr uint32_t MQ_Q = 0;                      // 128 rows x 256 B (two 16 KB halves)
-constexpr uint32_t MQ_K = 32768;                  // 2 stages x 32 KB
-constexpr uint32_t MQ_V = 98304;                  // 2 stages x 32 KB
-constexpr uint32_t MQ_BIAS = 163840;              // 2 buffers of staged diagonals
+constexpr uint32_t MQ_K = 32768;                  // 2 stages x 16 KB (two 64-row d halves)
+constexpr uint32_t MQ_V = 65536;                  // 2 stages x 16 KB
+constexpr uint32_t MQ_BIAS = 98304;               // 2 buffers of staged diagonals
 constexpr uint32_t MQ_BAR = MQ_BIAS + 2 * kMqBiasBuf * 4;
 constexpr int kMqSmem = MQ_BAR + 256 + 1024;
 
@@ -66,7 +67,7 @@ struct DecodeMqArgs {
     int S, Q, Hq, Hkv, G, max_blocks, num_blocks, window, d_max, splits;
 };
 
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, 2)
 decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const DecodeMqArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -88,7 +89,7 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int klo = (a.window > 0) ? max(0, L - Q - a.window + 1) : 0;
     int ta = 0, tb = 0;
     if (!bad_len) {
-        const int t_lo = klo >> 7, t_hi = (L - 1) >> 7;
+        const int t_lo = klo / kMqTile, t_hi = (L - 1) / kMqTile;
         const int per = (t_hi - t_lo + a.splits) / a.splits;
         ta = min(t_hi + 1, t_lo + split * per);
         tb = min(t_hi + 1, ta + per);
@@ -104,7 +105,7 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         fence_mbar_init();
     }
     if (warp == 5) {
-        tmem_alloc(tmem_slot, 512);
+        tmem_alloc(tmem_slot, 256);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -124,20 +125,20 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const int h = kvh * G + g;
         const int ipos = L - Q + qi;  // this row's query position
         const uint32_t tl = tbase + ((uint32_t)(warp * 32) << 16);
-        const uint32_t o_col = tl + 256;
+        const uint32_t o_col = tl + 128;
         const float scale = 0.08838834764831845f;  // 1/sqrt(128)
         const float kLog2e = 1.4426950408889634f;
         const float kTau = 5.545177444479562f;     // 8 ln 2
         const int W = a.window, Dm = a.d_max;
         float m_ref = -INFINITY, l = 0.f;
-        const int o_rd = Q - 1 - qi, sh = o_rd & 3;  // start of this row in its head's diagonal
-        const int span = Q + 127 + 3;                // staged values per head
+        const int o_rd = Q - 1 - qi;     // start of this row in its head's diagonal
+        const int span = Q + kMqTile - 1;  // staged values per head
         bool dead = bad_len;
         // diagonal of head g for key tile k: R[kk] = bias[h_g, clamp(L-1-j0-kk, 0, d_max)]
-        // (row qi reads R[Q-1-qi + c] for column c), as 4 copies shifted by
-        // 0..3 floats; thread t holds elements t, t+128, ... of the G x span
-        // values, fetched one tile ahead and stored under the next barrier
-        constexpr int kPer = (8 * (10 + 130) + 127) / 128;  // values per thread, G <= 8, Q <= 10
+        // (row qi reads R[Q-1-qi + c] for column c); thread t holds elements
+        // t, t+128, ... of the G x span values, fetched one tile ahead and
+        // stored under the next barrier
+        constexpr int kPer = (8 * (10 + kMqTile - 1) + 127) / 128;  // G <= 8, Q <= 10
         float nxt[kPer];
         // this thread's (head, offset) pairs, the same for every tile (-1: none)
         int egg[kPer], ekk[kPer];
@@ -148,7 +149,7 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             ekk[i] = e < G * span ? e % span : 0;
         }
         auto fetch = [&](int k) {
-            const int top = L - 1 - (ta + k) * 128;
+            const int top = L - 1 - (ta + k) * kMqTile;
 #pragma unroll
             for (int i = 0; i < kPer; ++i)
                 if (egg[i] >= 0)
@@ -158,20 +159,16 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         auto stage = [&](int k) {
             float *bb = (float *)(smem + MQ_BIAS) + (k & 1) * kMqBiasBuf;
 #pragma unroll
-            for (int i = 0; i < kPer; ++i) {
-                if (egg[i] < 0) continue;
-#pragma unroll
-                for (int s4 = 0; s4 < 4; ++s4)
-                    if (ekk[i] >= s4) bb[egg[i] * kMqHead + s4 * kMqCopy + ekk[i] - s4] = nxt[i];
-            }
+            for (int i = 0; i < kPer; ++i)
+                if (egg[i] >= 0) bb[egg[i] * kMqHead + ekk[i]] = nxt[i];
         };
         if (nt > 0) {
             fetch(0);
             stage(0);
         }
         for (int k = 0; k < nt; ++k) {
-            const int j0 = (ta + k) * 128;
-            float *bb = (float *)(smem + MQ_BIAS) + (k & 1) * kMqBiasBuf;
+            const int j0 = (ta + k) * kMqTile;
+            const float *bb = (const float *)(smem + MQ_BIAS) + (k & 1) * kMqBiasBuf;
             named_bar_sync(1, 128);  // tile k's diagonals are staged; tile k-1's reads are done
             if (k + 1 < nt) fetch(k + 1);
             if (!live) {
@@ -185,30 +182,30 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 continue;  // keep stepping through the group barrier
             }
             tc_fence_after();
-            const uint32_t s_col = tl + (k & 1) * 128;
-            uint32_t sr[128];
+            const uint32_t s_col = tl + (k & 1) * kMqTile;
+            uint32_t sr[64];
             tmem_ld32(s_col + 0, sr + 0);
             tmem_ld32(s_col + 32, sr + 32);
-            tmem_ld32(s_col + 64, sr + 64);
-            tmem_ld32(s_col + 96, sr + 96);
             tmem_wait_ld();
             // columns this row may see: ipos - j0 - c in [0, W)
             const int dist0 = ipos - j0;
-            const int cmax = rv ? min(127, dist0) : -1;
+            const int cmax = rv ? min(kMqTile - 1, dist0) : -1;
             const int cmin = (W > 0) ? max(0, dist0 - W + 1) : 0;
-            const bool full = cmin == 0 && cmax == 127;
-            const float4 *rp = (const float4 *)(bb + g * kMqHead + sh * kMqCopy + (o_rd - sh));
-            float x[128];
+            const bool full = cmin == 0 && cmax == kMqTile - 1;
+            const float *rb = bb + g * kMqHead + o_rd;
+            float x[64];
             float m8[8];
 #pragma unroll
             for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
             const f32x2 sc2 = pk2(scale, scale);
             auto logits = [&](auto masked) {
 #pragma unroll
-                for (int cb = 0; cb < 4; ++cb) {
+                for (int cb = 0; cb < 2; ++cb) {
                     float4 b4[8];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) b4[j] = rp[cb * 8 + j];
+                    for (int j = 0; j < 8; ++j)
+                        b4[j] = make_float4(rb[32 * cb + 4 * j], rb[32 * cb + 4 * j + 1],
+                                            rb[32 * cb + 4 * j + 2], rb[32 * cb + 4 * j + 3]);
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const int c = 32 * cb + 4 * j;
@@ -244,9 +241,9 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             {
                 const f32x2 l2e2 = pk2(kLog2e, kLog2e), mneg2 = pk2(mneg, mneg);
                 f32x2 acc[4] = {0ull, 0ull, 0ull, 0ull};
-                uint32_t pk[64];
+                uint32_t pk[32];
 #pragma unroll
-                for (int c = 0; c < 64; ++c) {
+                for (int c = 0; c < 32; ++c) {
                     const f32x2 tt = ffma2(pk2(x[2 * c], x[2 * c + 1]), l2e2, mneg2);
                     float t0, t1;
                     upk2(tt, t0, t1);
@@ -254,8 +251,7 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     acc[c & 3] = fadd2(acc[c & 3], pk2(p0, p1));
                     pk[c] = pack_bf16(p0, p1);
                 }
-                tmem_st32(s_col + 0, pk + 0);
-                tmem_st32(s_col + 32, pk + 32);
+                tmem_st32(s_col, pk);
                 const f32x2 s01 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
                 float la, lb;
                 upk2(s01, la, lb);
@@ -338,20 +334,21 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         for (int k = 0; k < nt; ++k) {
             const int st = k & 1;
             const uint32_t ph = ((k >> 1) & 1) ^ 1;
-            int blk = a.block_table[(long)s * a.max_blocks + ta + k];
+            int blk = a.block_table[(long)s * a.max_blocks + (ta + k) / 2];
             if (blk < 0 || blk >= a.num_blocks) {
                 report_status(a.status, INKLING_STATUS_BAD_BLOCK);
                 blk = 0;  // keep the pipeline running on a valid block
             }
-            const int row = (blk * a.Hkv + kvh) * 128;
+            const int n = ta + k;  // key tile: half n % 2 of cache block n / 2
+            const int row = (blk * a.Hkv + kvh) * 128 + (n & 1) * kMqTile;
             if (!mbar_wait(&bar[M_KEMPTY + st], ph, abort_flag, a.status)) break;
-            mbar_arrive_expect_tx(&bar[M_KFULL + st], 32768);
-            tma_load_2d(smem + MQ_K + st * 32768, &tm_k, &bar[M_KFULL + st], 0, row);
-            tma_load_2d(smem + MQ_K + st * 32768 + 16384, &tm_k, &bar[M_KFULL + st], 64, row);
+            mbar_arrive_expect_tx(&bar[M_KFULL + st], 16384);
+            tma_load_2d(smem + MQ_K + st * 16384, &tm_k, &bar[M_KFULL + st], 0, row);
+            tma_load_2d(smem + MQ_K + st * 16384 + 8192, &tm_k, &bar[M_KFULL + st], 64, row);
             if (!mbar_wait(&bar[M_VEMPTY + st], ph, abort_flag, a.status)) break;
-            mbar_arrive_expect_tx(&bar[M_VFULL + st], 32768);
-            tma_load_2d(smem + MQ_V + st * 32768, &tm_v, &bar[M_VFULL + st], 0, row);
-            tma_load_2d(smem + MQ_V + st * 32768 + 16384, &tm_v, &bar[M_VFULL + st], 64, row);
+            mbar_arrive_expect_tx(&bar[M_VFULL + st], 16384);
+            tma_load_2d(smem + MQ_V + st * 16384, &tm_v, &bar[M_VFULL + st], 0, row);
+            tma_load_2d(smem + MQ_V + st * 16384 + 8192, &tm_v, &bar[M_VFULL + st], 64, row);
             ++issued;
         }
         // drain: every load issued has landed before the block may exit
@@ -362,24 +359,25 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
     } else if (warp == 5 && lane == 0) {
         // ================================================ MMA issuer ==
-        const uint32_t id_qk = idesc_bf16(128, 128, 0, 0);
+        const uint32_t id_qk = idesc_bf16(128, kMqTile, 0, 0);
         const uint32_t id_pv = idesc_bf16(128, 128, 0, 1);
         auto issue_qk = [&](int k) {
             const int st = k & 1;
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
-                const uint64_t ad = sw128_desc(sb + MQ_Q + koff, 16, 1024);
-                const uint64_t bd = sw128_desc(sb + MQ_K + st * 32768 + koff, 16, 1024);
-                umma_ss(tbase + (k & 1) * 128, ad, bd, id_qk, ks > 0 ? 1u : 0u);
+                const uint64_t ad =
+                    sw128_desc(sb + MQ_Q + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+                const uint64_t bd =
+                    sw128_desc(sb + MQ_K + st * 16384 + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+                umma_ss(tbase + (k & 1) * kMqTile, ad, bd, id_qk, ks > 0 ? 1u : 0u);
             }
         };
         auto issue_pv = [&](int k) {
             const int st = k & 1;
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint64_t bd = sw128_desc(sb + MQ_V + st * 32768 + ks * 2048, 16384, 1024);
-                umma_ts(tbase + 256, tbase + (k & 1) * 128 + ks * 8, bd, id_pv,
+            for (int ks = 0; ks < kMqTile / 16; ++ks) {
+                const uint64_t bd = sw128_desc(sb + MQ_V + st * 16384 + ks * 2048, 8192, 1024);
+                umma_ts(tbase + 128, tbase + (k & 1) * kMqTile + ks * 8, bd, id_pv,
                         (k > 0 || ks > 0) ? 1u : 0u);
             }
         };
@@ -413,7 +411,7 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     __syncthreads();
     if (warp == 5) {
         tc_fence_after();
-        tmem_dealloc(tbase, 512);
+        tmem_dealloc(tbase, 256);
     }
 }
 

@@ -89,8 +89,31 @@ attn_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     const int ulo = lo[0];
     const int uhi = ok[1] ? hi[1] : hi[0];
 
+    // tile loads into this CTA's shared memory, completing on its own barriers
+    const int krow = 64 * (int)rank;
+    auto load_k = [&](int n, int st) {
+        mbar_arrive_expect_tx(&bar[K_RAW + st], 16384 + 2048);
+        for (int hf = 0; hf < 2; ++hf) {
+            tma_load_4d(smem + PK + st * 16384 + hf * 8192, &tm_k64, &bar[K_RAW + st], hf * 64,
+                        n * 128 + krow, kvh, b);
+            tma_load_4d(smem + PKH + st * 2048 + hf * 1024, &tm_kh, &bar[K_RAW + st], hf * 64,
+                        n * 128 + krow - 8, kvh, b);
+        }
+    };
+    auto load_v = [&](int n, int st) {
+        mbar_arrive_expect_tx(&bar[V_RAW + st], 16384 + 1024);
+        tma_load_4d(smem + PV + st * 16384, &tm_v, &bar[V_RAW + st], 64 * (int)rank, n * 128, kvh,
+                    b);
+        tma_load_4d(smem + PVH + st * 1024, &tm_vh, &bar[V_RAW + st], 64 * (int)rank,
+                    n * 128 - 8, kvh, b);
+    };
+    const int preload = min(kPS, uhi - ulo + 1);  // key/value tiles loaded during setup
+
     // ---- setup: barriers and the paired tensor-memory allocation must exist in
-    // both CTAs before either CTA signals the other
+    // both CTAs before either CTA signals the other.  The query tiles and the
+    // first kPS key/value tiles only involve this CTA's barriers, so the thread
+    // that initialises them starts those loads at once, under the allocation
+    // and the cluster barrier.
     if (threadIdx.x == 0) {
         for (int i = 0; i < NBAR; ++i) {
             uint32_t cnt = 1;
@@ -100,6 +123,16 @@ attn_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
         *abort_flag = 0;
         fence_mbar_init();
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&bar[Q_FULL], 65536);
+        for (int t = 0; t < 2; ++t)
+            for (int hf = 0; hf < 2; ++hf)
+                tma_load_4d(smem + PQ + t * 32768 + hf * 16384, &tm_q, &bar[Q_FULL], hf * 64,
+                            r0[t], h, b);
+        for (int i = 0; i < preload; ++i) {
+            load_k(ulo + i, i);
+            load_v(ulo + i, i);
+        }
     }
     if (warp == 13) {
         tmem_alloc_pair(tmem_slot, 512);
@@ -164,33 +197,18 @@ attn_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
             tma_prefetch_desc(&tm_kh);
             tma_prefetch_desc(&tm_v);
             tma_prefetch_desc(&tm_vh);
-            mbar_arrive_expect_tx(&bar[Q_FULL], 65536);
-            for (int t = 0; t < 2; ++t)
-                for (int hf = 0; hf < 2; ++hf)
-                    tma_load_4d(smem + PQ + t * 32768 + hf * 16384, &tm_q, &bar[Q_FULL], hf * 64,
-                                r0[t], h, b);
+            // the query tiles and the first kPS key/value tiles went out during setup
             if (rank == 1 && mbar_wait(&bar[Q_FULL], 0, abort_flag, a.status))
                 mbar_arrive_cta(&bar[Q_PEER], 0);
-            int kis = 0, vis = 0;  // key / value tile loads issued
-            const int krow = 64 * (int)rank;
-            for (int n = ulo; n <= uhi; ++n) {
+            int kis = preload, vis = preload;  // key / value tile loads issued
+            for (int n = ulo + preload; n <= uhi; ++n) {
                 const int it = n - ulo, st = it % kPS;
                 const uint32_t ph = ((it / kPS) & 1) ^ 1;
                 if (!mbar_wait(&bar[K_EMPTY + st], ph, abort_flag, a.status)) break;
-                mbar_arrive_expect_tx(&bar[K_RAW + st], 16384 + 2048);
-                for (int hf = 0; hf < 2; ++hf) {
-                    tma_load_4d(smem + PK + st * 16384 + hf * 8192, &tm_k64, &bar[K_RAW + st],
-                                hf * 64, n * 128 + krow, kvh, b);
-                    tma_load_4d(smem + PKH + st * 2048 + hf * 1024, &tm_kh, &bar[K_RAW + st],
-                                hf * 64, n * 128 + krow - 8, kvh, b);
-                }
+                load_k(n, st);
                 ++kis;
                 if (!mbar_wait(&bar[V_EMPTY + st], ph, abort_flag, a.status)) break;
-                mbar_arrive_expect_tx(&bar[V_RAW + st], 16384 + 1024);
-                tma_load_4d(smem + PV + st * 16384, &tm_v, &bar[V_RAW + st], 64 * (int)rank,
-                            n * 128, kvh, b);
-                tma_load_4d(smem + PVH + st * 1024, &tm_vh, &bar[V_RAW + st], 64 * (int)rank,
-                            n * 128 - 8, kvh, b);
+                load_v(n, st);
                 ++vis;
             }
             // drain: every load issued has landed before the block may exit
