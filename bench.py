@@ -43,7 +43,6 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # Set an entry to None when its kernel changes until it is captured again.
 MEASURED_TRAFFIC = {
     "prefill_swa_b4_t8192": 4 * 268.33e6,  # B1 capture x 4 batches
-    "decode_swa_s64": 1.049 * 1061945344,  # 16-sequence capture: traffic / KV bytes = 1.049
 }
 
 
