@@ -221,6 +221,10 @@ class ChunkStep:
         self.out = torch.empty_like(self.t["q"])
         self.flops = spec.flops
         self.launches = 2
+        mib = lambda x: x.numel() * x.element_size() / 2**20
+        cache = mib(self.t["k_cache"]) + mib(self.t["v_cache"])
+        self.l2_note = (f"inputs larger than L2 (q {mib(self.t['q']):.0f} MiB, "
+                        f"K/V cache {cache:.0f} MiB)")
 
     def run_append(self, stream=None):
         import relative_bias_sliding_b200 as ink
@@ -549,7 +553,7 @@ def run_chunk(args, chk, dist, rank, world, local, device):
                          "peak_source": f"{peak_src} bf16_tflops_sustained"},
             "chunk": {"sconv_append_ms": app_ms, "attn_prefill_paged_ms": attn_ms},
             "config": {"workload": chk.spec.name, "parallelism": f"replica per GPU x{world}",
-                       "l2": "inputs larger than L2 (q 256 MiB, cache 1 GiB)"},
+                       "l2": chk.l2_note},
             "e2e": None, "clocks": clocks.summary()}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, desc, thr = oracle_chunk_sample(chk.spec, args.cpu_seconds)

@@ -136,6 +136,11 @@ WORKLOADS = {
     # 2048-token chunk (the sliding-window prefill's shape, cut in chunks)
     "prefill_chunked_swa_b4_c2048": ChunkSpec("prefill_chunked_swa_b4_c2048", 4, 6144, 2048, 64,
                                               8, 128, 4096, 4096, 1.0, 5),
+    # the sliding-window prefill's shape (B4, T8192, window 4096) taken as one
+    # chunk over an empty cache: sconv append into the paged cache, then the
+    # paged prefill (zero sconv history)
+    "prefill_paged_swa_b4_t8192": ChunkSpec("prefill_paged_swa_b4_t8192", 4, 0, 8192, 64, 8,
+                                            128, 4096, 4096, 1.0, 1),
     # output sconv over the sliding-window prefill's attention output
     "sconv_out_b4_t8192": SconvOutSpec("sconv_out_b4_t8192", 4, 8192, 64 * 128, 6),
     # smaller cuts of the same workloads for profiler captures (still larger
@@ -241,7 +246,8 @@ def make_chunk(spec: ChunkSpec, device="cpu"):
     """Chunked-prefill step inputs: packed chunk queries q [B*chunk, Hq, d] with
     row offsets cu_q, the chunk's raw keys/values [B, chunk, Hkv, d], taps,
     bias, sconv states, and a paged cache whose prefix slots hold N(0, 1)
-    post-sconv rows (the append overwrites the chunk's slots)."""
+    post-sconv rows (the append overwrites the chunk's slots).  With no
+    prefix the sconv states are zero."""
     g = _generator(device, spec.seed)
     B, Hq, Hkv, d, n = spec.B, spec.Hq, spec.Hkv, spec.d, spec.chunk
     C = Hkv * d
@@ -254,6 +260,9 @@ def make_chunk(spec: ChunkSpec, device="cpu"):
                        dtype=torch.float32) * spec.bias_std
     k_state = _normal_bf16(g, (B, 3, C), device)
     v_state = _normal_bf16(g, (B, 3, C), device)
+    if spec.prefix == 0:  # an empty sequence has zero sconv history
+        k_state.zero_()
+        v_state.zero_()
     L = spec.prefix + n
     nb = (L + BLOCK - 1) // BLOCK
     perm = torch.randperm(B * nb, generator=g, device=device).to(torch.int32)

@@ -129,14 +129,16 @@ def test_chunked_prefill_reports_short_length():
     assert status.item() & 4   # INKLING_STATUS_BAD_LENGTH: 10 new tokens, length 5
 
 
-def test_chunked_workload_sampled_rows(oracle_mod):
-    """The chunked-prefill bench workload (4 sequences, 6144-token prefix,
-    2048-token chunk, window 4096): GPU append + paged prefill; sampled
-    (row, head) pairs against the oracle's append + paged attention of the
-    same rows (query r at position prefix + r)."""
+@pytest.mark.parametrize("name", ["prefill_chunked_swa_b4_c2048", "prefill_paged_swa_b4_t8192"])
+def test_chunked_workload_sampled_rows(oracle_mod, name):
+    """The chunked-prefill bench workloads (4 sequences with a 6144-token
+    prefix and a 2048-token chunk; 4 empty sequences taking 8192 tokens;
+    window 4096): GPU append + paged prefill; sampled (row, head) pairs against
+    the oracle's append + paged attention of the same rows (query r at
+    position prefix + r)."""
     need_gpu()
     from relative_bias_sliding_b200.inputs import make_chunk
-    spec = WORKLOADS_CHUNK["prefill_chunked_swa_b4_c2048"]
+    spec = WORKLOADS_CHUNK[name]
     t = make_chunk(spec)
     host = {k: v.clone() for k, v in t.items()}
     dev = {k: v.cuda() for k, v in t.items()}
