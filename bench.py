@@ -35,6 +35,9 @@ if ROOT not in sys.path:
 METRIC = "prefill TFLOP/s and decode KV GB/s on 1 B200, as % of BF16/HBM roofline"
 DEFAULT_PREFILL = "prefill_swa_b4_t8192"
 DEFAULT_DECODE = "decode_swa_s64"
+# the same sliding-window prefill shape through the paged cache: sconv append
+# of all keys/values, then the paged prefill (timed after the main step)
+DEFAULT_VIA_CACHE = "prefill_paged_swa_b4_t8192"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one
@@ -42,7 +45,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # scaled by the units processed (profiles/ holds the summaries and commands).
 # Set an entry to None when its kernel changes until it is captured again.
 MEASURED_TRAFFIC = {
-    "prefill_swa_b4_t8192": 4 * 268.33e6,  # B1 capture x 4 batches
+    "prefill_swa_b4_t8192": 4 * 268.13e6,  # B1 capture x 4 batches
 }
 
 
@@ -513,8 +516,10 @@ def run_reference(args):
     return 0
 
 
-def run_chunk(args, chk, dist, rank, world, local, device):
-    """Bench line of a chunked-prefill workload (device-timed; no e2e leg)."""
+def time_chunk(args, chk, dist, local, device, clocks_dir):
+    """Warm up, then time ``args.steps`` chunk steps (append, paged prefill) on
+    one stream; returns (step ms, append ms, attention ms) as the max over
+    ranks, and the clock sampler."""
     import torch
     stream = torch.cuda.Stream(device)
     fns = [chk.run_append, chk.run_attn]
@@ -524,7 +529,7 @@ def run_chunk(args, chk, dist, rank, world, local, device):
     stream.synchronize()
     barrier(dist, device)
     torch.cuda.synchronize()
-    with ClockSampler(local, args.clocks_log_dir) as clocks:
+    with ClockSampler(local, clocks_dir) as clocks:
         barrier(dist, device)
         torch.cuda.synchronize()
         t_start = torch.cuda.Event(enable_timing=True)
@@ -536,10 +541,16 @@ def run_chunk(args, chk, dist, rank, world, local, device):
         torch.cuda.synchronize()
         barrier(dist, device)
     step_ms = t_start.elapsed_time(t_end) / args.steps
-    per_fn = max_over_ranks(dist, per_fn, device)
+    app_ms, attn_ms = max_over_ranks(dist, per_fn, device)
     step_ms = max_over_ranks(dist, [step_ms], device)[0]
+    return step_ms, app_ms, attn_ms, clocks
+
+
+def run_chunk(args, chk, dist, rank, world, local, device):
+    """Bench line of a chunked-prefill workload (device-timed; no e2e leg)."""
+    step_ms, app_ms, attn_ms, clocks = time_chunk(args, chk, dist, local, device,
+                                                  args.clocks_log_dir)
     peaks, peak_src = load_peaks()
-    app_ms, attn_ms = per_fn
     tflops = chk.flops / ((app_ms + attn_ms) * 1e-3) / 1e12 * world
     kern = chk.flops / (attn_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
@@ -731,6 +742,24 @@ def main():
                            "ms_per_step": ms2, "h2d_bytes_per_step": h2d2,
                            "d2h_bytes_per_step": d2h2}
     line["clocks"] = clocks.summary()
+
+    if not args.workload:
+        # the same prefill shape through the paged cache (sconv append of all
+        # keys/values, then the paged prefill), timed on its own after the step
+        via = ChunkStep(WORKLOADS[DEFAULT_VIA_CACHE], device)
+        v_step, v_app, v_attn, v_clocks = time_chunk(args, via, dist, local, device, None)
+        v_kern = via.flops / (v_attn * 1e-3) / 1e12
+        line["prefill_via_cache"] = {
+            "workload": via.spec.name, "value": via.flops / ((v_app + v_attn) * 1e-3) / 1e12 * world,
+            "unit": "TFLOP/s", "ms_per_step": v_step, "sconv_append_ms": v_app,
+            "attn_prefill_paged_ms": v_attn, "gpu_launches": args.steps * via.launches,
+            "roofline": {"bound": "tensor", "kernel": "attn_prefill_paged_kernel",
+                         "achieved": v_kern, "peak": peaks["bf16_tflops_sustained"],
+                         "unit": "TFLOP/s", "frac": v_kern / peaks["bf16_tflops_sustained"],
+                         "traffic": MEASURED_TRAFFIC.get(via.spec.name),
+                         "peak_source": f"{peak_src} bf16_tflops_sustained"},
+            "clocks": v_clocks.summary()}
+        del via
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         if pre:
