@@ -41,11 +41,12 @@ DEFAULT_VIA_CACHE = "prefill_paged_swa_b4_t8192"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one
-# ncu capture of the current kernels on a smaller cut of the same workload,
-# scaled by the units processed (profiles/ holds the summaries and commands).
-# Set an entry to None when its kernel changes until it is captured again.
+# ncu capture of the current kernels on the workload itself (one launch after
+# 3 warm-up launches; profiles/ holds the summaries and commands).  Remove an
+# entry when its kernel changes until it is captured again.
 MEASURED_TRAFFIC = {
-    "prefill_swa_b4_t8192": 4 * 268.13e6,  # B1 capture x 4 batches
+    "prefill_swa_b4_t8192": 676_643_840 + 501_745_152,
+    "prefill_paged_swa_b4_t8192": 675_873_792 + 496_937_216,
 }
 
 

@@ -69,13 +69,16 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // ---- work item: heaviest query blocks first, heads of one kv group adjacent
-    const int bh = a.B * a.Hq;
-    const int qb = a.nqb - 1 - (int)(blockIdx.x / bh);
-    const int b = (int)(blockIdx.x % bh) / a.Hq;
-    const int h = (int)(blockIdx.x % bh) % a.Hq;
+    // ---- work item: CTAs run grouped by (sequence, kv head), so the CTAs
+    // resident at one time read the same keys/values (they stay in L2); inside
+    // a group the heaviest query blocks come first.
     const int G = a.Hq / a.Hkv;
-    const int kvh = h / G;
+    const int per_group = a.nqb * G;
+    const int grp = (int)(blockIdx.x / per_group), rem = (int)(blockIdx.x % per_group);
+    const int b = grp / a.Hkv;
+    const int kvh = grp % a.Hkv;
+    const int qb = a.nqb - 1 - rem / G;
+    const int h = kvh * G + rem % G;
     int r0[2], lo[2], hi[2];
     bool ok[2];
 #pragma unroll

@@ -78,12 +78,16 @@ attn_prefill_paged_kernel(const __grid_constant__ CUtensorMap tm_q,
     const PrefillArgs &a = g.pa;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // ---- work item: later (longer) query blocks first
-    const int sh = g.S * a.Hq;
-    const int qb = g.nqb - 1 - (int)(blockIdx.x / sh);
-    const int s = (int)(blockIdx.x % sh) / a.Hq;
-    const int h = (int)(blockIdx.x % sh) % a.Hq;
-    const int kvh = h / (a.Hq / a.Hkv);
+    // ---- work item: CTAs run grouped by (sequence, kv head), so the CTAs
+    // resident at one time read the same cache blocks (they stay in L2); inside
+    // a group the later (longer) query blocks come first.
+    const int G = a.Hq / a.Hkv;
+    const int per_group = g.nqb * G;
+    const int grp = (int)(blockIdx.x / per_group), rem = (int)(blockIdx.x % per_group);
+    const int s = grp / a.Hkv;
+    const int kvh = grp % a.Hkv;
+    const int qb = g.nqb - 1 - rem / G;
+    const int h = kvh * G + rem % G;
     const int q_begin = g.cu_q[s];
     const int n = g.cu_q[s + 1] - q_begin;  // new tokens (query rows) of this sequence
     const int L = g.seq_lens[s];

@@ -67,14 +67,17 @@ attn_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();  // 0 issues the MMAs
 
-    // ---- work item: heaviest query blocks first; a cluster = 2 heads of one kv group
+    // ---- work item: a cluster = 2 heads of one kv group.  Clusters run
+    // grouped by (sequence, kv head), so the clusters resident at one time read
+    // the same keys/values (they stay in L2); inside a group the heaviest query
+    // blocks come first.
     const int G = a.Hq / a.Hkv, GP = G / 2;
-    const int per_qb = a.B * a.Hkv * GP;
+    const int per_group = a.nqb * GP;
     const int cid = (int)(blockIdx.x >> 1);
-    const int qb = a.nqb - 1 - cid / per_qb;
-    const int rem = cid % per_qb;
-    const int b = rem / (a.Hkv * GP);
-    const int kvh = (rem / GP) % a.Hkv;
+    const int grp = cid / per_group, rem = cid % per_group;
+    const int b = grp / a.Hkv;
+    const int kvh = grp % a.Hkv;
+    const int qb = a.nqb - 1 - rem / GP;
     const int h = kvh * G + 2 * (rem % GP) + (int)rank;
     int r0[2], lo[2], hi[2];
     bool ok[2];
