@@ -2,9 +2,10 @@
 // 2-SM tensor-core MMAs (tcgen05 cta_group::2), for GQA groups of even size.
 //
 // Same layer and numerics (vLLM Recipes "thinkingmachines/Inkling", Overview:
-// "Attention" and "Short convolution").  A 2-CTA cluster takes two query heads
-// of one kv group and the same 256-row query block, so both CTAs walk the same
-// key/value tiles.  Each MMA is M = 256 (128 query rows from each CTA's shared
+// "Attention" and "Short convolution").  A 2-CTA cluster takes query heads of
+// one kv group over the same query rows (4 heads x 128 rows when the group
+// size is a multiple of 4, else 2 heads x 256 rows), so both CTAs walk the
+// same key/value tiles.  Each MMA is M = 256 (128 query rows from each CTA's shared
 // memory, accumulators in each CTA's own tensor memory) and reads the B
 // operand half from each CTA:
 //   QK^T: N = 128 keys; CTA r holds keys 64r..64r+63 of the tile (all of d);
@@ -25,7 +26,7 @@
 namespace inkling {
 
 constexpr int kPS = 3;                          // key/value pipeline stages
-constexpr uint32_t PQ = 0;                      // 2 query tiles x 32 KB (this CTA's head)
+constexpr uint32_t PQ = 0;                      // 2 query tiles x 32 KB
 constexpr uint32_t PK = 65536;                  // kPS x 16 KB: this CTA's 64 keys x 128 d
 constexpr uint32_t PV = PK + kPS * 16384;       // kPS x 16 KB: 128 keys x this CTA's 64 d
 constexpr uint32_t PKH = PV + kPS * 16384;      // kPS x 2 KB: 8 history rows x 2 halves
@@ -67,23 +68,30 @@ attn_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();  // 0 issues the MMAs
 
-    // ---- work item: a cluster = 2 heads of one kv group.  Clusters run
-    // grouped by (sequence, kv head), so the clusters resident at one time read
-    // the same keys/values (they stay in L2); inside a group the heaviest query
-    // blocks come first.
-    const int G = a.Hq / a.Hkv, GP = G / 2;
-    const int per_group = a.nqb * GP;
+    // ---- work item.  When the GQA group size is a multiple of 4, a cluster
+    // takes 4 heads of one kv group over the same 128 query rows: CTA r holds
+    // heads 4q+2r and 4q+2r+1 as its two query tiles, so both tiles walk the
+    // same key range.  Otherwise it takes 2 heads (one per CTA) over 256 rows,
+    // two 128-row tiles per CTA whose key ranges differ by one tile at each end.
+    // Clusters run grouped by (sequence, kv head), so the clusters resident at
+    // one time read the same keys/values (they stay in L2); inside a group the
+    // heaviest query blocks come first.
+    const int G = a.Hq / a.Hkv;
+    const bool quad = (G & 3) == 0;
+    const int per_qb = quad ? G / 4 : G / 2;  // clusters per (kv head, query block)
+    const int per_group = a.nqb * per_qb;
     const int cid = (int)(blockIdx.x >> 1);
     const int grp = cid / per_group, rem = cid % per_group;
     const int b = grp / a.Hkv;
     const int kvh = grp % a.Hkv;
-    const int qb = a.nqb - 1 - rem / GP;
-    const int h = kvh * G + 2 * (rem % GP) + (int)rank;
-    int r0[2], lo[2], hi[2];
+    const int qb = a.nqb - 1 - rem / per_qb;
+    const int hsel = rem % per_qb;
+    int hd[2], r0[2], lo[2], hi[2];
     bool ok[2];
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
-        r0[t] = qb * kQRows + t * 128;
+        hd[t] = quad ? kvh * G + 4 * hsel + 2 * (int)rank + t : kvh * G + 2 * hsel + (int)rank;
+        r0[t] = quad ? qb * 128 : qb * 256 + t * 128;
         ok[t] = r0[t] < a.T;
         const int rmax = min(r0[t] + 127, a.T - 1);
         hi[t] = rmax >> 7;
@@ -131,7 +139,7 @@ attn_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int t = 0; t < 2; ++t)
             for (int hf = 0; hf < 2; ++hf)
                 tma_load_4d(smem + PQ + t * 32768 + hf * 16384, &tm_q, &bar[Q_FULL], hf * 64,
-                            r0[t], h, b);
+                            r0[t], hd[t], b);
         for (int i = 0; i < preload; ++i) {
             load_k(ulo + i, i);
             load_v(ulo + i, i);
@@ -153,12 +161,12 @@ attn_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int t = warp >> 2;
         if (ok[t])
             softmax_role(a, (float *)(smem + PBIAS) + t * 2 * kBiasBuf, &bar[S_FULL], &bar[O_DONE],
-                         abort_flag, tbase, t, h, r0[t], a.T, lo[t], hi[t], 3 + t,
+                         abort_flag, tbase, t, hd[t], r0[t], a.T, lo[t], hi[t], 3 + t,
                          [&](int tt) {
                              __syncwarp();
                              if (lane == 0) mbar_arrive_cta_relaxed(&bar[P_FULL + tt], 0);
                          },
-                         TmaStoreEpilogue{a, smem + PQ + t * 32768, &tm_out, b, h, r0[t], 3 + t});
+                         TmaStoreEpilogue{a, smem + PQ + t * 32768, &tm_out, b, hd[t], r0[t], 3 + t});
     } else if (warp < 12) {
         // ==================== sconv of this CTA's halves: warps 8-9 keys, 10-11 values ==
         setmaxnreg_dec80();
@@ -333,8 +341,10 @@ cudaError_t launch_attn_prefill_pair(const inkling_prefill_params &p, const CUte
     a.Hkv = p.num_kv_heads;
     a.window = p.window;
     a.d_max = p.d_max;
-    a.nqb = (p.seq_len + kQRows - 1) / kQRows;
-    const long clusters = (long)a.B * a.Hkv * (a.Hq / a.Hkv / 2) * a.nqb;
+    const int G = a.Hq / a.Hkv;
+    const bool quad = (G & 3) == 0;  // 4 heads x 128 rows per cluster, else 2 heads x 256 rows
+    a.nqb = quad ? (p.seq_len + 127) / 128 : (p.seq_len + 255) / 256;
+    const long clusters = (long)a.B * a.Hkv * (quad ? G / 4 : G / 2) * a.nqb;
     if (clusters == 0) return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(attn_prefill_pair_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem);

@@ -49,6 +49,8 @@ def test_prefill_tiny_workload_all_rows(oracle_mod):
     (1, 1000, 16, 2, 300, 50),   # window + clip, ragged
     (1, 520, 8, 1, 1, 8),        # window of one key (self only)
     (3, 257, 8, 4, 256, 300),    # query block boundary + 1
+    (1, 600, 12, 2, 200, 300),   # G = 6: two heads x 256 rows per CTA pair
+    (2, 400, 12, 3, 0, 400),     # G = 4, three kv heads: four heads x 128 rows per pair
 ])
 def test_prefill_ragged_and_masks(oracle_mod, B, T, Hq, Hkv, W, D_max):
     need_gpu()
@@ -63,6 +65,7 @@ def test_prefill_ragged_and_masks(oracle_mod, B, T, Hq, Hkv, W, D_max):
 @pytest.mark.parametrize("B,T,Hq,Hkv,W", [
     (1, 2560, 32, 4, 0),      # 160 CTA pairs: more than fit on the GPU at once
     (2, 2500, 32, 4, 1000),   # 320 pairs, ragged tail, window not a multiple of a tile
+    (1, 2900, 24, 4, 700),    # G = 6 (two heads x 256 rows per pair), 132 pairs, ragged
 ])
 def test_prefill_several_waves_all_rows(oracle_mod, B, T, Hq, Hkv, W):
     """More (head pair, query block) CTA pairs than fit on the GPU at once, with
