@@ -85,6 +85,8 @@ def _chunked(seqs, w_k, w_v, bias, chunks, window, Hkv, extra_blocks=3, seed=0):
     (8, 1, 0, 2000),     # G = 8, full causal
     (6, 2, 300, 256),    # G = 3, window, clip inside the band
     (4, 4, 128, 1000),   # G = 1, window of exactly one tile
+    (4, 2, 500, 600),    # G = 2: two heads x 128 rows per block, window, clip
+    (12, 2, 0, 1500),    # G = 6: three head pairs per kv head, full causal
 ])
 def test_chunked_prefill_equals_whole_sequence_oracle(oracle_mod, Hq, Hkv, window, D_max):
     need_gpu()
