@@ -19,13 +19,13 @@
 // all MMAs.  The odd CTA's threads report to the even CTA's mbarriers:
 // converted halves (K/V ready), their P tiles (per warp) and their Q load.
 // Commits are multicast to the same barrier offset in both CTAs, so each CTA's
-// softmax and producer wait on local barriers.  Key/value stages: 3.  No TMA
+// softmax and producer wait on local barriers.  Key/value stages: 4.  No TMA
 // load uses multicast.
 #include "prefill_common.cuh"
 
 namespace inkling {
 
-constexpr int kPS = 3;                          // key/value pipeline stages
+constexpr int kPS = 4;                          // key/value pipeline stages
 constexpr uint32_t PQ = 0;                      // 2 query tiles x 32 KB
 constexpr uint32_t PK = 65536;                  // kPS x 16 KB: this CTA's 64 keys x 128 d
 constexpr uint32_t PV = PK + kPS * 16384;       // kPS x 16 KB: 128 keys x this CTA's 64 d
@@ -39,17 +39,18 @@ enum {
     Q_FULL = 0,
     Q_PEER = 1,   // even CTA: the odd CTA's query tiles have landed
     K_RAW = 2,    // +stage
-    V_RAW = 5,
-    K_READY = 8,  // even CTA: both halves converted (64 + 64 arrivals)
-    V_READY = 11,
-    K_EMPTY = 14,
-    V_EMPTY = 17,
-    S_FULL = 20,  // +query tile
-    P_FULL = 22,  // even CTA: 4 warps of each CTA
-    O_DONE = 24,
-    DRAIN = 26,
-    NBAR = 27
+    V_RAW = K_RAW + kPS,
+    K_READY = V_RAW + kPS,  // even CTA: both halves converted (64 + 64 arrivals)
+    V_READY = K_READY + kPS,
+    K_EMPTY = V_READY + kPS,
+    V_EMPTY = K_EMPTY + kPS,
+    S_FULL = V_EMPTY + kPS,  // +query tile
+    P_FULL = S_FULL + 2,  // even CTA: 4 warps of each CTA
+    O_DONE = P_FULL + 2,
+    DRAIN = O_DONE + 2,
+    NBAR = DRAIN + 1
 };
+static_assert(kPairSmem <= 232448, "shared memory per block");
 
 __global__ void __launch_bounds__(512, 1)
 attn_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
