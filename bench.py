@@ -174,6 +174,26 @@ class PrefillStep:
         ink.attn_prefill(t["q"], t["k_raw"], t["v_raw"], t["w_k"], t["w_v"], t["bias"],
                          window=self.spec.window, out=self.out, stream=stream)
 
+    def add_cache(self, device):
+        """Paged cache, block table and sconv states for the cache-filling
+        variant of the same prefill (blocks in a random order)."""
+        import torch
+        B, T, Hkv = self.spec.B, self.spec.T, self.spec.Hkv
+        nb = (T + 127) // 128
+        g = torch.Generator(device=device).manual_seed(self.spec.seed + 100)
+        self.bt = torch.randperm(B * nb, generator=g, device=device).to(torch.int32).reshape(B, nb)
+        self.kc = torch.zeros((B * nb, Hkv, 128, 128), dtype=torch.bfloat16, device=device)
+        self.vc = torch.zeros_like(self.kc)
+        self.ks = torch.zeros((B, 3, Hkv * 128), dtype=torch.bfloat16, device=device)
+        self.vs = torch.zeros_like(self.ks)
+
+    def run_fill(self, stream=None):
+        import relative_bias_sliding_b200 as ink
+        t = self.t
+        ink.attn_prefill(t["q"], t["k_raw"], t["v_raw"], t["w_k"], t["w_v"], t["bias"],
+                         window=self.spec.window, out=self.out, stream=stream, k_cache=self.kc,
+                         v_cache=self.vc, block_table=self.bt, k_state=self.ks, v_state=self.vs)
+
     launches = 1
 
 
@@ -517,6 +537,23 @@ def run_reference(args):
     return 0
 
 
+def time_loop_only(args, fns, dist, device):
+    """Warm up, then time ``args.steps`` passes over ``fns`` on one stream;
+    per-callable mean ms, max over ranks."""
+    import torch
+    stream = torch.cuda.Stream(device)
+    for _ in range(args.warmup):
+        for f in fns:
+            f(stream)
+    stream.synchronize()
+    barrier(dist, device)
+    torch.cuda.synchronize()
+    per_fn = timed_loop(args.steps, fns, stream)
+    torch.cuda.synchronize()
+    barrier(dist, device)
+    return max_over_ranks(dist, per_fn, device)
+
+
 def time_chunk(args, chk, dist, local, device, clocks_dir):
     """Warm up, then time ``args.steps`` chunk steps (append, paged prefill) on
     one stream; returns (step ms, append ms, attention ms) as the max over
@@ -745,6 +782,15 @@ def main():
     line["clocks"] = clocks.summary()
 
     if not args.workload:
+        # the same fused prefill also writing the paged cache and the sconv
+        # state in the same pass, timed on its own after the step
+        pre.add_cache(device)
+        f_ms = time_loop_only(args, [pre.run_fill], dist, device)[0]
+        line["prefill_fills_cache"] = {
+            "workload": pre.spec.name, "value": pre.flops / (f_ms * 1e-3) / 1e12 * world,
+            "unit": "TFLOP/s", "ms_per_step": f_ms, "gpu_launches": args.steps,
+            "cache_bytes_written": pre.spec.B * pre.spec.T * pre.spec.Hkv * 128 * 2 * 2,
+            "plain_ms_per_step": per_fn[0]}
         # the same prefill shape through the paged cache (sconv append of all
         # keys/values, then the paged prefill), timed on its own after the step
         via = ChunkStep(WORKLOADS[DEFAULT_VIA_CACHE], device)

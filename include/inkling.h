@@ -128,6 +128,18 @@ inkling_status inkling_sconv_kv(const inkling_sconv_params *p, inkling_stream_t 
  * inkling_sconv_kv would write them.  Logits use scale 1/sqrt(128) on q.k and
  * add bias[h, min(i-j, d_max)] unscaled; softmax and accumulation are fp32,
  * probabilities enter the P.V product as bf16, the output is rounded to bf16.
+ *
+ * Optional cache fill in the same pass (the sconv state is managed like the
+ * KV cache of a sliding-window layer, Overview, "Short convolution"): when
+ * k_cache, v_cache and block_table are given, the post-sconv keys and values
+ * of tokens 0..T-1 of sequence b are also written to the paged cache, token t
+ * at slot t%128 of block block_table[b, t/128], bit for bit what
+ * inkling_sconv_kv writes when it appends the T tokens to an empty sequence.
+ * Slots at positions >= T are not touched.  When k_state and v_state are also
+ * given, they receive the new sconv state: the raw rows T-3..T-1 (zero where
+ * negative), oldest first, so that inkling_sconv_kv continues the sequence.
+ * A block id outside [0, num_blocks) sets INKLING_STATUS_BAD_BLOCK in *status
+ * and that tile is not written.  With B = 0 or T = 0 nothing is written.
  * -------------------------------------------------------------------------- */
 typedef struct {
     const void *q;        /* device [B, T, Hq, d] bf16 */
@@ -146,6 +158,14 @@ typedef struct {
     int32_t head_dim;     /* d, must be 128 */
     int32_t window;       /* 0 = full causal, else keys with i-j < window */
     int32_t d_max;        /* bias table has d_max+1 entries per head, d_max >= 0 */
+    /* optional cache fill (all NULL = none; k_cache, v_cache and block_table together) */
+    void *k_cache;              /* device [num_blocks, Hkv, 128, d] bf16, or NULL */
+    void *v_cache;              /* device [num_blocks, Hkv, 128, d] bf16, or NULL */
+    const int32_t *block_table; /* device [B, max_blocks] int32, or NULL */
+    int32_t max_blocks;         /* columns of block_table, max_blocks*128 >= T */
+    int32_t num_blocks;         /* blocks in the cache pool */
+    void *k_state;              /* device [B, 3, Hkv*d] bf16 out, or NULL (with v_state) */
+    void *v_state;              /* device [B, 3, Hkv*d] bf16 out, or NULL (with k_state) */
 } inkling_prefill_params;
 
 inkling_status inkling_attn_prefill(const inkling_prefill_params *p, inkling_stream_t stream);

@@ -51,7 +51,8 @@ class PrefillParams(ctypes.Structure):
     _fields_ = [("q", _P), ("k_raw", _P), ("v_raw", _P), ("w_k", _P), ("w_v", _P), ("bias", _P),
                 ("out", _P), ("lse", _P), ("status", _P), ("batch", _I), ("seq_len", _I),
                 ("num_q_heads", _I), ("num_kv_heads", _I), ("head_dim", _I), ("window", _I),
-                ("d_max", _I)]
+                ("d_max", _I), ("k_cache", _P), ("v_cache", _P), ("block_table", _P),
+                ("max_blocks", _I), ("num_blocks", _I), ("k_state", _P), ("v_state", _P)]
 
 
 class SconvOutParams(ctypes.Structure):
@@ -176,8 +177,14 @@ def sconv_kv(k_new, v_new, w_k, w_v, k_state, v_state, k_cache, v_cache, block_t
 
 
 def attn_prefill(q, k_raw, v_raw, w_k, w_v, bias, window=0, out=None, lse=None, status=None,
-                 stream=None):
-    """Prefill attention with fused sconv; returns ``out`` [B, T, Hq, d] bf16."""
+                 stream=None, k_cache=None, v_cache=None, block_table=None, k_state=None,
+                 v_state=None):
+    """Prefill attention with fused sconv; returns ``out`` [B, T, Hq, d] bf16.
+
+    With ``k_cache``, ``v_cache`` [num_blocks, Hkv, 128, d] and ``block_table``
+    [B, max_blocks] the same pass writes the post-sconv keys/values of tokens
+    0..T-1 into the paged cache; with ``k_state``, ``v_state`` [B, 3, Hkv*d]
+    it writes the new sconv state."""
     bf, f32 = torch.bfloat16, torch.float32
     _dev(q, bf, "q", 4), _dev(k_raw, bf, "k_raw", 4), _dev(v_raw, bf, "v_raw", 4)
     B, T, Hq, d = q.shape
@@ -202,8 +209,27 @@ def attn_prefill(q, k_raw, v_raw, w_k, w_v, bias, window=0, out=None, lse=None, 
         if lse.shape != (B, Hq, T):
             raise ValueError("lse must be [B, Hq, T]")
     _dev(status, torch.int32, "status")
+    max_blocks = num_blocks = 0
+    if k_cache is not None or v_cache is not None or block_table is not None:
+        if k_cache is None or v_cache is None or block_table is None:
+            raise ValueError("k_cache, v_cache and block_table go together")
+        for n, t in (("k_cache", k_cache), ("v_cache", v_cache)):
+            _dev(t, bf, n, 4)
+            if t.shape[1:] != (Hkv, BLOCK_SIZE, d):
+                raise ValueError(f"{n} must be [num_blocks, {Hkv}, {BLOCK_SIZE}, {d}]")
+        _dev(block_table, torch.int32, "block_table", 2)
+        if block_table.shape[0] != B:
+            raise ValueError("block_table must be [B, max_blocks]")
+        max_blocks, num_blocks = block_table.shape[1], k_cache.shape[0]
+    for n, t in (("k_state", k_state), ("v_state", v_state)):
+        if t is not None:
+            _dev(t, bf, n, 3)
+            if t.shape != (B, 3, Hkv * d):
+                raise ValueError(f"{n} must be [{B}, 3, {Hkv * d}]")
     p = PrefillParams(_ptr(q), _ptr(k_raw), _ptr(v_raw), _ptr(w_k), _ptr(w_v), _ptr(bias),
-                      _ptr(out), _ptr(lse), _ptr(status), B, T, Hq, Hkv, d, int(window), d_max)
+                      _ptr(out), _ptr(lse), _ptr(status), B, T, Hq, Hkv, d, int(window), d_max,
+                      _ptr(k_cache), _ptr(v_cache), _ptr(block_table), max_blocks, num_blocks,
+                      _ptr(k_state), _ptr(v_state))
     _check(load_library().inkling_attn_prefill(ctypes.byref(p), _stream(stream)))
     return out
 

@@ -249,6 +249,22 @@ inkling_status inkling_attn_prefill(const inkling_prefill_params *p, inkling_str
     if (!aligned16(p->q) || !aligned16(p->k_raw) || !aligned16(p->v_raw) || !aligned16(p->w_k) ||
         !aligned16(p->w_v) || !aligned16(p->out))
         return fail(INKLING_ERR_INVALID, "q, k_raw, v_raw, taps and out must be 16-byte aligned");
+    if (p->k_cache || p->v_cache || p->block_table) {
+        if (!p->k_cache || !p->v_cache || !p->block_table)
+            return fail(INKLING_ERR_INVALID, "k_cache, v_cache and block_table go together");
+        if (!aligned16(p->k_cache) || !aligned16(p->v_cache))
+            return fail(INKLING_ERR_INVALID, "caches must be 16-byte aligned");
+        if (p->max_blocks < 1 || p->num_blocks < 1)
+            return fail(INKLING_ERR_INVALID, "max_blocks and num_blocks must be >= 1");
+        if ((long)p->max_blocks * 128 < p->seq_len)
+            return fail(INKLING_ERR_INVALID, "max_blocks * 128 < seq_len");
+        if ((long)p->num_blocks * p->num_kv_heads * 128 >= (1L << 31))
+            return fail(INKLING_ERR_UNSUPPORTED, "cache pool rows exceed 2^31");
+    }
+    if ((p->k_state != nullptr) != (p->v_state != nullptr))
+        return fail(INKLING_ERR_INVALID, "k_state and v_state go together");
+    if (p->k_state && (!aligned16(p->k_state) || !aligned16(p->v_state)))
+        return fail(INKLING_ERR_INVALID, "states must be 16-byte aligned");
     inkling_status st = check_device(nullptr);
     if (st != INKLING_OK) return st;
 

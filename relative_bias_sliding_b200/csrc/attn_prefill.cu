@@ -53,13 +53,18 @@ enum {
     B_COUNT = 20
 };
 
+// kFill: also write the post-sconv keys/values to the paged cache and the new
+// sconv state (a separate instantiation, so the plain prefill keeps its
+// registers).
+template <bool kFill>
 __global__ void __launch_bounds__(512, 1)
 attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_kh,
                     const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_vh,
-                    const __grid_constant__ CUtensorMap tm_out, const PrefillArgs a) {
+                    const __grid_constant__ CUtensorMap tm_out, const PrefillArgs a,
+                    const FillArgs f) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sb = smem_u32(smem);
@@ -134,6 +139,9 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
         uint64_t *ready = &bar[is_v ? B_VREADY : B_KREADY];
         const uint32_t tiles = sb + (is_v ? SM_V : SM_K);
         const uint32_t hists = sb + (is_v ? SM_VH : SM_KH);
+        // with a cache to fill, the block of the kv group's first head writes
+        // the key tiles this query block owns (2qb up to its last tile)
+        const bool writer = kFill && h == kvh * G && f.k_cache != nullptr;
         bool dead = false;
         int it = 0;
         for (int n = ulo; n <= uhi; ++n, ++it) {
@@ -146,12 +154,19 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
             // thread v: column v % 16, rows 32 (v / 16) .. +32 of the 128-row tile
             sconv_rows(tiles + st * 32768, hists + st * 2048, 16384, w, v & 15, 32 * (v >> 4), 32,
                        bar_id, 64);
+            if (kFill && writer && n >= 2 * qb) {
+                uint16_t *gdst = cache_rows(f, a, is_v ? f.v_cache : f.k_cache, b, kvh, n, 0, 8 * (v & 15));
+                if (gdst) store_rows(tiles + st * 32768, 16384, v & 15, 32 * (v >> 4), 32, gdst, a.T - n * 128);
+            }
             fence_proxy_async_smem();
             mbar_arrive(&ready[st]);
         }
     } else {
         setmaxnreg_dec64();
-        if (warp == 12 && lane == 0) {
+        if (kFill && warp == 14 && h == kvh * G && f.k_state && uhi == (a.T - 1) >> 7) {
+            // the new sconv state, by the block that owns the last key tile
+            write_sconv_state(f, a, b, kvh, lane);
+        } else if (warp == 12 && lane == 0) {
             // ============================================== TMA producer ==
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
@@ -280,7 +295,7 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
 
 cudaError_t launch_attn_prefill(const inkling_prefill_params &p, const CUtensorMap *maps,
                                 cudaStream_t stream) {
-    PrefillArgs a;
+    PrefillArgs a = {};
     a.w_k = p.w_k;
     a.w_v = p.w_v;
     a.bias = p.bias;
@@ -293,14 +308,26 @@ cudaError_t launch_attn_prefill(const inkling_prefill_params &p, const CUtensorM
     a.Hkv = p.num_kv_heads;
     a.window = p.window;
     a.d_max = p.d_max;
+    FillArgs f = {};
+    f.k_cache = (uint16_t *)p.k_cache;
+    f.v_cache = (uint16_t *)p.v_cache;
+    f.block_table = p.block_table;
+    f.max_blocks = p.max_blocks;
+    f.num_blocks = p.num_blocks;
+    f.k_state = (uint16_t *)p.k_state;
+    f.v_state = (uint16_t *)p.v_state;
+    f.k_raw = (const uint16_t *)p.k_raw;
+    f.v_raw = (const uint16_t *)p.v_raw;
     a.nqb = (p.seq_len + kQRows - 1) / kQRows;
     const long grid = (long)a.B * a.Hq * a.nqb;
     if (grid == 0) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(attn_prefill_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kPrefillSmem);
+    const bool fill = f.k_cache != nullptr || f.k_state != nullptr;
+    auto kernel = fill ? attn_prefill_kernel<true> : attn_prefill_kernel<false>;
+    cudaError_t e =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPrefillSmem);
     if (e != cudaSuccess) return e;
-    attn_prefill_kernel<<<(unsigned)grid, 512, kPrefillSmem, stream>>>(maps[0], maps[1], maps[2],
-                                                                      maps[3], maps[4], maps[5], a);
+    kernel<<<(unsigned)grid, 512, kPrefillSmem, stream>>>(maps[0], maps[1], maps[2], maps[3],
+                                                         maps[4], maps[5], a, f);
     return cudaGetLastError();
 }
 

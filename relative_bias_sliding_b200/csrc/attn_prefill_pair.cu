@@ -52,13 +52,18 @@ enum {
 };
 static_assert(kPairSmem <= 232448, "shared memory per block");
 
+// kFill: also write the post-sconv keys/values to the paged cache and the new
+// sconv state (a separate instantiation, so the plain prefill keeps its
+// registers).
+template <bool kFill>
 __global__ void __launch_bounds__(512, 1)
 attn_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k64,
                          const __grid_constant__ CUtensorMap tm_kh,
                          const __grid_constant__ CUtensorMap tm_v,
                          const __grid_constant__ CUtensorMap tm_vh,
-                    const __grid_constant__ CUtensorMap tm_out, const PrefillArgs a) {
+                    const __grid_constant__ CUtensorMap tm_out, const PrefillArgs a,
+                    const FillArgs f) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sb = smem_u32(smem);
@@ -186,6 +191,10 @@ attn_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
         const uint32_t tiles = sb + (is_v ? PV : PK);
         const uint32_t hists = sb + (is_v ? PVH : PKH);
         const uint32_t hist_stage = is_v ? 1024 : 2048;
+        // with a cache to fill, the first cluster of the (sequence, kv head)
+        // for this query block writes the key tiles it owns: quad ? qb : 2qb
+        // up to its last tile (each CTA its converted half)
+        const bool writer = kFill && hsel == 0 && f.k_cache != nullptr;
         bool dead = false;
         int it = 0;
         for (int n = ulo; n <= uhi; ++n, ++it) {
@@ -197,12 +206,21 @@ attn_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
             }
             sconv_rows(tiles + st * 16384, hists + st * hist_stage, 8192, w, col, row0, 16, bar_id,
                        64);
+            if (kFill && writer && n >= (quad ? qb : 2 * qb)) {
+                const int krow = is_v ? 0 : 64 * (int)rank;  // token row of this CTA's tile row 0
+                uint16_t *gdst = cache_rows(f, a, is_v ? f.v_cache : f.k_cache, b, kvh, n, krow, ch0);
+                if (gdst) store_rows(tiles + st * 16384, 8192, col, row0, 16, gdst, a.T - n * 128 - krow);
+            }
             fence_proxy_async_smem();
             mbar_arrive_cta(&ready[st], 0);
         }
     } else {
         setmaxnreg_dec64();
-        if (warp == 12 && lane == 0) {
+        if (kFill && warp == 14 && rank == 0 && hsel == 0 && f.k_state &&
+            uhi == (a.T - 1) >> 7) {
+            // the new sconv state, by the block that owns the last key tile
+            write_sconv_state(f, a, b, kvh, lane);
+        } else if (warp == 12 && lane == 0) {
             // ============================================== TMA producer ==
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k64);
@@ -329,7 +347,7 @@ attn_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
 
 cudaError_t launch_attn_prefill_pair(const inkling_prefill_params &p, const CUtensorMap *maps,
                                      cudaStream_t stream) {
-    PrefillArgs a;
+    PrefillArgs a = {};
     a.w_k = p.w_k;
     a.w_v = p.w_v;
     a.bias = p.bias;
@@ -342,13 +360,25 @@ cudaError_t launch_attn_prefill_pair(const inkling_prefill_params &p, const CUte
     a.Hkv = p.num_kv_heads;
     a.window = p.window;
     a.d_max = p.d_max;
+    FillArgs f = {};
+    f.k_cache = (uint16_t *)p.k_cache;
+    f.v_cache = (uint16_t *)p.v_cache;
+    f.block_table = p.block_table;
+    f.max_blocks = p.max_blocks;
+    f.num_blocks = p.num_blocks;
+    f.k_state = (uint16_t *)p.k_state;
+    f.v_state = (uint16_t *)p.v_state;
+    f.k_raw = (const uint16_t *)p.k_raw;
+    f.v_raw = (const uint16_t *)p.v_raw;
     const int G = a.Hq / a.Hkv;
     const bool quad = (G & 3) == 0;  // 4 heads x 128 rows per cluster, else 2 heads x 256 rows
     a.nqb = quad ? (p.seq_len + 127) / 128 : (p.seq_len + 255) / 256;
     const long clusters = (long)a.B * a.Hkv * (quad ? G / 4 : G / 2) * a.nqb;
     if (clusters == 0) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(attn_prefill_pair_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem);
+    const bool fill = f.k_cache != nullptr || f.k_state != nullptr;
+    auto kernel = fill ? attn_prefill_pair_kernel<true> : attn_prefill_pair_kernel<false>;
+    cudaError_t e =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
@@ -362,8 +392,8 @@ cudaError_t launch_attn_prefill_pair(const inkling_prefill_params &p, const CUte
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, attn_prefill_pair_kernel, maps[0], maps[1], maps[2], maps[3],
-                           maps[4], maps[5], a);
+    e = cudaLaunchKernelEx(&cfg, kernel, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5],
+                           a, f);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

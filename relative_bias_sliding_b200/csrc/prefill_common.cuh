@@ -23,6 +23,48 @@ struct PrefillArgs {
     int B, T, Hq, Hkv, window, d_max, nqb;
 };
 
+// Optional outputs of the prefill (a kernel argument of its own, so that the
+// plain prefill's argument block and registers are those without them):
+// post-sconv keys/values into the paged cache [num_blocks, Hkv, 128, 128]
+// through block_table [B, max_blocks], and the new sconv state
+// [B, 3, Hkv*128] (the last 3 raw rows of k_raw / v_raw).
+struct FillArgs {
+    uint16_t *k_cache, *v_cache, *k_state, *v_state;
+    const int32_t *block_table;
+    const uint16_t *k_raw, *v_raw;
+    int max_blocks, num_blocks;
+};
+
+// Where the converted rows of key tile n go in the paged cache: the address of
+// tile row 0 (token n*128 + row_base) at channel `ch` of kv head kvh.  A block
+// id outside the pool is reported and gives nullptr (nothing is written).
+INK_DEV uint16_t *cache_rows(const FillArgs &f, const PrefillArgs &a, uint16_t *cache, int b,
+                             int kvh, int n, int row_base, int ch) {
+    const int blk = __ldg(f.block_table + (long)b * f.max_blocks + n);
+    if (blk < 0 || blk >= f.num_blocks) {
+        report_status(a.status, INKLING_STATUS_BAD_BLOCK);
+        return nullptr;
+    }
+    return cache + (((long)blk * a.Hkv + kvh) * 128 + row_base) * 128 + ch;
+}
+
+// New sconv state of (sequence b, kv head kvh) after a prefill of T tokens
+// from zero history: rows T-3..T-1 of the raw keys/values (zero where the
+// index is negative), for both K and V.  One warp; 16-byte copies.
+INK_DEV void write_sconv_state(const FillArgs &f, const PrefillArgs &a, int b, int kvh, int lane) {
+    const long C = (long)a.Hkv * 128;
+    for (int k = lane; k < 2 * 3 * 16; k += 32) {
+        const bool v = k >= 48;
+        const int m = (k % 48) >> 4, chunk = k & 15;
+        const int t = a.T - 3 + m;
+        const uint16_t *raw = v ? f.v_raw : f.k_raw;
+        uint16_t *state = v ? f.v_state : f.k_state;
+        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        if (t >= 0) val = *(const uint4 *)(raw + (((long)b * a.T + t) * a.Hkv + kvh) * 128 + chunk * 8);
+        *(uint4 *)(state + ((long)b * 3 + m) * C + (long)kvh * 128 + chunk * 8) = val;
+    }
+}
+
 // Register split per warpgroup: 2 x 128 softmax threads at 184, 128 sconv
 // threads at 80, 128 producer/MMA/idle threads at 64: 47104 + 10240 + 8192 =
 // 65536 = 512 threads x the 128 registers the kernels launch with (ptxas
@@ -92,6 +134,22 @@ INK_DEV void sconv_rows(uint32_t tile, uint32_t hist, uint32_t half_bytes, const
         sts128(addr, make_uint4(o[0], o[1], o[2], o[3]));
 #pragma unroll
         for (int p = 0; p < 4; ++p) { h3[p] = h2[p]; h2[p] = h1[p]; h1[p] = x[p]; }
+    }
+}
+
+// Copy of the rows [row0, row0 + nrows) of column `c` that this thread has just
+// converted (same layout as sconv_rows) to the paged cache: tile row r goes to
+// gdst + r*128 (gdst = tile row 0 at this column's channels) when r < gvalid.
+// Only the calling thread's own shared-memory writes are read, so no barrier
+// is needed; a separate pass keeps the transform's registers unchanged.
+INK_DEV void store_rows(uint32_t tile, uint32_t half_bytes, int c, int row0, int nrows,
+                        uint16_t *gdst, int gvalid) {
+    const uint32_t tb = tile + (c >> 3) * half_bytes;
+    const int cc = c & 7;
+    for (int i = 0; i < nrows; ++i) {
+        const int r = row0 + i;
+        if (r >= gvalid) break;
+        *(uint4 *)(gdst + (long)r * 128) = lds128(tb + r * 128 + ((cc ^ (r & 7)) << 4));
     }
 }
 

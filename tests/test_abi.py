@@ -49,6 +49,8 @@ int main(void) {{
          sizeof(inkling_prefill_params), sizeof(inkling_decode_params),
          sizeof(inkling_prefill_paged_params));
   F(inkling_sconv_params, num_blocks) F(inkling_prefill_params, d_max)
+  F(inkling_prefill_params, k_cache) F(inkling_prefill_params, max_blocks)
+  F(inkling_prefill_params, v_state)
   F(inkling_decode_params, num_splits) F(inkling_decode_params, status)
   F(inkling_decode_params, q_len) F(inkling_prefill_paged_params, cu_q)
   F(inkling_prefill_paged_params, max_q) F(inkling_prefill_paged_params, d_max)
@@ -65,6 +67,8 @@ int main(void) {{
     assert int(out["decode"]) == ctypes.sizeof(binding.DecodeParams)
     assert int(out["inkling_sconv_params num_blocks"]) == binding.SconvParams.num_blocks.offset
     assert int(out["inkling_prefill_params d_max"]) == binding.PrefillParams.d_max.offset
+    for m in ("k_cache", "max_blocks", "v_state"):
+        assert int(out["inkling_prefill_params " + m]) == getattr(binding.PrefillParams, m).offset
     assert int(out["inkling_decode_params num_splits"]) == binding.DecodeParams.num_splits.offset
     assert int(out["inkling_decode_params status"]) == binding.DecodeParams.status.offset
     assert int(out["inkling_decode_params q_len"]) == binding.DecodeParams.q_len.offset
@@ -100,6 +104,27 @@ def test_host_validation_rejects_before_launch(lib):
     p.batch = 0
     assert lib.inkling_attn_prefill(ctypes.byref(p), None) == binding.INKLING_OK  # empty: no-op
     assert lib.inkling_attn_prefill(None, None) == binding.INKLING_ERR_INVALID
+
+    # the optional cache fill: argument checks come before any device access
+    # (the addresses below are never dereferenced)
+    fake = ctypes.c_void_p(1 << 20)
+    p.batch = 1
+    for f in ("q", "k_raw", "v_raw", "w_k", "w_v", "bias", "out"):
+        setattr(p, f, fake)
+    p.k_cache = fake
+    assert lib.inkling_attn_prefill(ctypes.byref(p), None) == binding.INKLING_ERR_INVALID
+    assert b"together" in lib.inkling_last_error()
+    p.v_cache, p.block_table, p.max_blocks, p.num_blocks = fake, fake, 0, 4
+    assert lib.inkling_attn_prefill(ctypes.byref(p), None) == binding.INKLING_ERR_INVALID
+    p.seq_len, p.max_blocks = 300, 2
+    assert lib.inkling_attn_prefill(ctypes.byref(p), None) == binding.INKLING_ERR_INVALID
+    assert b"max_blocks * 128" in lib.inkling_last_error()
+    p.max_blocks, p.k_state = 3, fake
+    assert lib.inkling_attn_prefill(ctypes.byref(p), None) == binding.INKLING_ERR_INVALID
+    assert b"k_state and v_state" in lib.inkling_last_error()
+    p.v_state = ctypes.c_void_p((1 << 20) + 8)
+    assert lib.inkling_attn_prefill(ctypes.byref(p), None) == binding.INKLING_ERR_INVALID
+    assert b"16-byte" in lib.inkling_last_error()
 
     d = binding.DecodeParams()
     d.num_seqs, d.num_q_heads, d.num_kv_heads, d.head_dim = 2, 64, 4, 128
