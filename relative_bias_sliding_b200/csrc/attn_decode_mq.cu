@@ -54,7 +54,8 @@ enum {
     M_PFULL = 11,   // +S buffer (128 arrivals)
     M_OREADY = 13,  // one phase per P.V issued
     M_DRAIN = 14,
-    M_COUNT = 15
+    M_ODONE = 15,   // the last P.V has completed (one phase)
+    M_COUNT = 16
 };
 
 struct DecodeMqArgs {
@@ -281,9 +282,11 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             mbar_arrive(&bar[M_PFULL + (k & 1)]);
             if (k + 1 < nt) stage(k + 1);
         }
-        // epilogue: the last P.V has completed
+        // epilogue: the last P.V has completed.  It has a one-phase barrier of
+        // its own: a parity wait on M_OREADY could match the phase of the P.V
+        // two tiles back if the one before it had not completed yet
         const bool have_o = live && !dead && nt > 0 &&
-                            mbar_wait_warp(&bar[M_OREADY], (nt - 1) & 1, abort_flag, a.status);
+                            mbar_wait_warp(&bar[M_ODONE], 0, abort_flag, a.status);
         if (have_o) tc_fence_after();
         uint32_t ob[128];
         if (have_o) {
@@ -401,6 +404,7 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 issue_pv(kp);
                 tc_commit(&bar[M_OREADY]);
                 tc_commit(&bar[M_VEMPTY + (kp & 1)]);
+                if (kp == nt - 1) tc_commit(&bar[M_ODONE]);
             }
         }
         // every MMA issued has completed before TMEM is released
