@@ -84,7 +84,7 @@ INK_DEV bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int3
     }
 }
 
-// Warp-uniform bounded wait: lane 0 spins, the verdict is broadcast, and on
+// Warp-uniform bounded wait: lane 0 spins, the outcome is broadcast, and on
 // success every lane re-observes the completed phase (acquire for its reads).
 INK_DEV bool mbar_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort,
                             int32_t *status) {
