@@ -38,6 +38,11 @@ DEFAULT_DECODE = "decode_swa_s64"
 # the same sliding-window prefill shape through the paged cache: sconv append
 # of all keys/values, then the paged prefill (timed after the main step)
 DEFAULT_VIA_CACHE = "prefill_paged_swa_b4_t8192"
+# the layer's other workloads, each timed after the step with its own roofline
+# and oracle timing: the tiny and the 32k full-causal prefill; multi-token
+# decode (9 draft tokens); 1M-token full-attention decode at batch 1 and 8
+EXTRA_PREFILL = ["prefill_tiny_b1_t256", "prefill_full_b1_t32768"]
+EXTRA_DECODE = ["decode_mtp9_swa_s64", "decode_full_1m_b1", "decode_full_1m_b8"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one
@@ -155,6 +160,31 @@ def load_peaks():
             d = json.load(f)
         return d, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+def tensor_roofline(achieved, kernel, traffic=None, clocks=None):
+    """Roofline object of a tensor-bound kernel.  The peak is the burst cuBLAS
+    bf16 figure: the kernels here run at the maximum SM clock without the power
+    cap (the `clocks` of the same line show it), so the burst figure, the
+    higher of the two measured peaks, is the one they are held to; the
+    fraction of the sustained (power-capped) figure is given beside it."""
+    peaks, src = load_peaks()
+    burst = peaks["bf16_tflops"]
+    sus = peaks.get("bf16_tflops_sustained", burst)
+    note = f"{src} bf16_tflops (burst)"
+    if clocks:
+        note += (f"; kernel timed at median {clocks.get('sm_mhz')} MHz of max "
+                 f"{clocks.get('sm_max_mhz')}, reasons {clocks.get('reasons')}")
+    return {"bound": "tensor", "kernel": kernel, "achieved": achieved, "peak": burst,
+            "unit": "TFLOP/s", "frac": achieved / burst, "traffic": traffic, "peak_source": note,
+            "frac_of_sustained": achieved / sus, "sustained_peak": sus}
+
+
+def hbm_roofline(achieved, kernel, traffic=None):
+    peaks, src = load_peaks()
+    return {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+            "peak_source": f"{src} hbm_gbs"}
 
 
 # ----------------------------------------------------------- GPU workload --
@@ -424,6 +454,37 @@ def oracle_decode_sample(spec, seconds, seed=0):
     return done_bytes / total_t / 1e9, desc, oracle.num_threads()
 
 
+def oracle_decode_long_sample(dec):
+    """Time the oracle's decode step on one whole sequence of a long-context
+    decode workload whose cache lives on the device: sequence 0's blocks are
+    copied to the host in order (K and V, 4 GiB at 1M tokens), then the sconv
+    append of its new token and the attention of all its query heads run on
+    the oracle.  Returns (KV GB/s, description, threads)."""
+    import numpy as np
+    import torch
+    import oracle
+    t, spec = dec.t, dec.spec
+    u = lambda x: x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    L = int(t["seq_lens"][0])
+    nb = (L + 127) // 128
+    ids = t["block_table"][0, :nb].long()
+    kc, vc = u(t["k_cache"][ids]).copy(), u(t["v_cache"][ids]).copy()
+    ks, vs = u(t["k_state"][:1]).copy(), u(t["v_state"][:1]).copy()
+    bt = np.arange(nb, dtype=np.int32)[None, :]
+    sl = np.array([L], np.int32)
+    q, kn, vn = u(t["q"][:1]), u(t["k_new"][:1]), u(t["v_new"][:1])
+    wk, wv, bias = (t[k].cpu().numpy() for k in ("w_k", "w_v", "bias"))
+    t0 = time.perf_counter()
+    oracle.sconv_append(kn, ks, wk, kc, bt, sl)
+    oracle.sconv_append(vn, vs, wv, vc, bt, sl)
+    oracle.decode_rows(q, kc, vc, bt, sl, bias, spec.window, spec.D_max)
+    dt = time.perf_counter() - t0
+    keys = min(L, spec.window) if spec.window > 0 else L
+    desc = (f"1 whole sequence of {spec.name} ({L} tokens, all {spec.Hq} heads, sconv append "
+            f"included), {dt:.1f} s")
+    return keys * spec.Hkv * spec.d * 4 / dt / 1e9, desc, oracle.num_threads()
+
+
 def oracle_chunk_sample(spec, seconds, seed=0):
     """Time the oracle's chunked-prefill step (sconv append of one sequence's
     chunk, then its chunk rows over the paged cache, all heads) on a bounded
@@ -588,18 +649,14 @@ def run_chunk(args, chk, dist, rank, world, local, device):
     """Bench line of a chunked-prefill workload (device-timed; no e2e leg)."""
     step_ms, app_ms, attn_ms, clocks = time_chunk(args, chk, dist, local, device,
                                                   args.clocks_log_dir)
-    peaks, peak_src = load_peaks()
     tflops = chk.flops / ((app_ms + attn_ms) * 1e-3) / 1e12 * world
     kern = chk.flops / (attn_ms * 1e-3) / 1e12
-    peak = peaks["bf16_tflops_sustained"]
     line = {"metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "gpu_launches": args.steps * chk.launches,
-            "roofline": {"bound": "tensor", "kernel": "attn_prefill_paged_kernel",
-                         "achieved": kern, "peak": peak, "unit": "TFLOP/s", "frac": kern / peak,
-                         "traffic": MEASURED_TRAFFIC.get(chk.spec.name),
-                         "peak_source": f"{peak_src} bf16_tflops_sustained"},
+            "roofline": tensor_roofline(kern, "attn_prefill_paged_kernel",
+                                        MEASURED_TRAFFIC.get(chk.spec.name), clocks.summary()),
             "chunk": {"sconv_append_ms": app_ms, "attn_prefill_paged_ms": attn_ms},
             "config": {"workload": chk.spec.name, "parallelism": f"replica per GPU x{world}",
                        "l2": chk.l2_note},
@@ -655,6 +712,70 @@ def run_sconv_out(args, spec, dist, rank, world, local, device):
     return 0
 
 
+def time_with_clocks(args, fns, dist, local, device, steps=None):
+    """Warm up, then time ``steps`` (default --steps) passes over ``fns`` on one
+    stream with the clocks sampled; per-callable mean ms (max over ranks), the
+    whole-pass ms, and the clock summary."""
+    import torch
+    steps = steps or args.steps
+    stream = torch.cuda.Stream(device)
+    for _ in range(args.warmup):
+        for f in fns:
+            f(stream)
+    stream.synchronize()
+    barrier(dist, device)
+    torch.cuda.synchronize()
+    with ClockSampler(local, args.clocks_log_dir) as clocks:
+        barrier(dist, device)
+        torch.cuda.synchronize()
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        per_fn = timed_loop(steps, fns, stream)
+        t_end.record(stream)
+        stream.synchronize()
+        torch.cuda.synchronize()
+        barrier(dist, device)
+    step_ms = t_start.elapsed_time(t_end) / steps
+    per_fn = max_over_ranks(dist, per_fn, device)
+    step_ms = max_over_ranks(dist, [step_ms], device)[0]
+    return per_fn, step_ms, clocks.summary()
+
+
+def prefill_object(args, pre, ms, step_ms, steps, world, clocks, with_cpu):
+    """Bench sub-object of one prefill workload (kernel time = step time: one
+    launch per step)."""
+    tflops = pre.flops / (ms * 1e-3) / 1e12
+    obj = {"workload": pre.spec.name, "value": tflops * world, "unit": "TFLOP/s",
+           "ms_per_step": step_ms, "steps": steps, "gpu_launches": steps,
+           "flops_per_step": pre.flops,
+           "roofline": tensor_roofline(tflops, "attn_prefill_pair_kernel",
+                                       MEASURED_TRAFFIC.get(pre.spec.name), clocks),
+           "clocks": clocks}
+    if with_cpu:
+        v, desc, thr = oracle_prefill_sample(pre.spec, args.cpu_seconds)
+        obj["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+                               "sample": desc}
+    return obj
+
+
+def decode_object(dec, app_ms, attn_ms, step_ms, steps, world, clocks):
+    """Bench sub-object of one decode workload: value = key/value bytes per
+    step over (sconv append + decode); the roofline is the decode kernels
+    alone."""
+    gbs = dec.kv_bytes / ((app_ms + attn_ms) * 1e-3) / 1e9
+    kern = dec.kv_bytes / (attn_ms * 1e-3) / 1e9
+    mq = dec.spec.n_new > 1
+    kernel = ("decode_mq_tc_kernel" if mq else "decode_split_kernel") + \
+        (" + decode_combine_kernel" if dec.splits > 1 else "")
+    return {"workload": dec.spec.name, "value": gbs * world, "unit": "GB/s",
+            "ms_per_step": step_ms, "steps": steps, "gpu_launches": steps * dec.launches,
+            "sconv_append_ms": app_ms, "attn_decode_ms": attn_ms, "num_splits": dec.splits,
+            "kv_bytes_per_step": dec.kv_bytes,
+            "roofline": hbm_roofline(kern, kernel, MEASURED_TRAFFIC.get(dec.spec.name)),
+            "clocks": clocks}
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -672,8 +793,8 @@ def main():
     ink.load_library()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    with_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
 
-    chk = None
     if args.workload:
         spec = WORKLOADS[args.workload]
         if isinstance(spec, SconvOutSpec):
@@ -685,33 +806,14 @@ def main():
     else:
         pre = PrefillStep(WORKLOADS[DEFAULT_PREFILL], device)
         dec = DecodeStep(WORKLOADS[DEFAULT_DECODE], device)
-    stream = torch.cuda.Stream(device)
     fns = []
     if pre:
         fns.append(pre.run)
     if dec:
         fns += [dec.run_append, dec.run_attn]
 
-    for _ in range(args.warmup):
-        for f in fns:
-            f(stream)
-    stream.synchronize()
-    barrier(dist, device)
-    torch.cuda.synchronize()
-    with ClockSampler(local, args.clocks_log_dir) as clocks:
-        barrier(dist, device)
-        torch.cuda.synchronize()
-        t_start = torch.cuda.Event(enable_timing=True)
-        t_end = torch.cuda.Event(enable_timing=True)
-        t_start.record(stream)
-        per_fn = timed_loop(args.steps, fns, stream)
-        t_end.record(stream)
-        stream.synchronize()
-        torch.cuda.synchronize()
-        barrier(dist, device)
-    step_ms = t_start.elapsed_time(t_end) / args.steps
-    per_fn = max_over_ranks(dist, per_fn, device)
-    step_ms = max_over_ranks(dist, [step_ms], device)[0]
+    per_fn, step_ms, clocks = time_with_clocks(args, fns, dist, local, device)
+    stream = torch.cuda.Stream(device)
 
     e2e = None
     if not args.no_e2e:
@@ -722,37 +824,23 @@ def main():
             e2e_parts.append(("dec",) + e2e_decode(dec, max(3, args.steps // 4), stream))
         e2e = e2e_parts
 
-    peaks, peak_src = load_peaks()
     line = {"metric": METRIC, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "gpu_launches": args.steps * sum(x.launches for x in (pre, dec) if x) * 1}
+            "gpu_launches": args.steps * sum(x.launches for x in (pre, dec) if x)}
     i = 0
     if pre:
         pre_ms = per_fn[0]
         i = 1
         tflops = pre.flops / (pre_ms * 1e-3) / 1e12 * world
-        peak = peaks["bf16_tflops_sustained"]
         line.update({"value": tflops, "unit": "TFLOP/s"})
-        line["roofline"] = {"bound": "tensor", "kernel": "attn_prefill_pair_kernel",
-                            "achieved": tflops / world, "peak": peak, "unit": "TFLOP/s",
-                            "frac": tflops / world / peak,
-                            "traffic": MEASURED_TRAFFIC.get(pre.spec.name),
-                            "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed "
-                                           f"inside a long step loop)"}
+        line["roofline"] = tensor_roofline(tflops / world, "attn_prefill_pair_kernel",
+                                           MEASURED_TRAFFIC.get(pre.spec.name), clocks)
     if dec:
         app_ms, attn_ms = per_fn[i], per_fn[i + 1]
-        gbs = dec.kv_bytes / ((app_ms + attn_ms) * 1e-3) / 1e9
-        kern_gbs = dec.kv_bytes / (attn_ms * 1e-3) / 1e9
-        dec_obj = {"workload": dec.spec.name, "value": gbs * world, "unit": "GB/s",
-                   "ms_per_step": app_ms + attn_ms, "sconv_append_ms": app_ms,
-                   "attn_decode_ms": attn_ms, "num_splits": dec.splits,
-                   "kv_bytes_per_step": dec.kv_bytes,
-                   "roofline": {"bound": "hbm", "kernel": "decode_split_kernel + combine",
-                                "achieved": kern_gbs, "peak": peaks["hbm_gbs"],
-                                "unit": "GB/s", "frac": kern_gbs / peaks["hbm_gbs"],
-                                "traffic": MEASURED_TRAFFIC.get(dec.spec.name),
-                                "peak_source": f"{peak_src} hbm_gbs"}}
+        dec_obj = decode_object(dec, app_ms, attn_ms, app_ms + attn_ms, args.steps, world,
+                                clocks)
+        del dec_obj["clocks"]
         if pre:
             line["decode"] = dec_obj
         else:
@@ -779,7 +867,7 @@ def main():
             line["e2e"] = {"value": dec.kv_bytes / (ms2 * 1e-3) / 1e9 * world, "unit": "GB/s",
                            "ms_per_step": ms2, "h2d_bytes_per_step": h2d2,
                            "d2h_bytes_per_step": d2h2}
-    line["clocks"] = clocks.summary()
+    line["clocks"] = clocks
 
     if not args.workload:
         # the same fused prefill also writing the paged cache and the sconv
@@ -796,26 +884,65 @@ def main():
         via = ChunkStep(WORKLOADS[DEFAULT_VIA_CACHE], device)
         v_step, v_app, v_attn, v_clocks = time_chunk(args, via, dist, local, device, None)
         v_kern = via.flops / (v_attn * 1e-3) / 1e12
+        vc = v_clocks.summary()
         line["prefill_via_cache"] = {
             "workload": via.spec.name, "value": via.flops / ((v_app + v_attn) * 1e-3) / 1e12 * world,
             "unit": "TFLOP/s", "ms_per_step": v_step, "sconv_append_ms": v_app,
             "attn_prefill_paged_ms": v_attn, "gpu_launches": args.steps * via.launches,
-            "roofline": {"bound": "tensor", "kernel": "attn_prefill_paged_kernel",
-                         "achieved": v_kern, "peak": peaks["bf16_tflops_sustained"],
-                         "unit": "TFLOP/s", "frac": v_kern / peaks["bf16_tflops_sustained"],
-                         "traffic": MEASURED_TRAFFIC.get(via.spec.name),
-                         "peak_source": f"{peak_src} bf16_tflops_sustained"},
-            "clocks": v_clocks.summary()}
+            "roofline": tensor_roofline(v_kern, "attn_prefill_paged_kernel",
+                                        MEASURED_TRAFFIC.get(via.spec.name), vc),
+            "clocks": vc}
         del via
+        if with_cpu:
+            # the oracle on the decode workload of the step
+            v, desc, thr = oracle_decode_sample(dec.spec, args.cpu_seconds)
+            line["decode"]["cpu_baseline"] = {"value": v, "unit": "GB/s", "cores": thr,
+                                              "kind": "oracle", "sample": desc}
+        del pre, dec
+        torch.cuda.empty_cache()
+        # the other workloads of the layer, each timed on its own with its
+        # roofline and the oracle timed beside it
+        for name in EXTRA_PREFILL:
+            p2 = PrefillStep(WORKLOADS[name], device)
+            steps = max(args.steps, 200) if p2.flops < 1e10 else args.steps
+            pf, pstep, pclk = time_with_clocks(args, [p2.run], dist, local, device, steps)
+            line[name] = prefill_object(args, p2, pf[0], pstep, steps, world, pclk, with_cpu)
+            del p2
+            torch.cuda.empty_cache()
+        for name in EXTRA_DECODE:
+            d2 = DecodeStep(WORKLOADS[name], device)
+            df, dstep, dclk = time_with_clocks(args, [d2.run_append, d2.run_attn], dist, local,
+                                               device)
+            obj = decode_object(d2, df[0], df[1], dstep, args.steps, world, dclk)
+            if with_cpu:
+                if d2.spec.L_min >= (1 << 16):
+                    v, desc, thr = oracle_decode_long_sample(d2)
+                else:
+                    v, desc, thr = oracle_decode_sample(d2.spec, args.cpu_seconds)
+                obj["cpu_baseline"] = {"value": v, "unit": "GB/s", "cores": thr,
+                                       "kind": "oracle", "sample": desc}
+            line[name] = obj
+            del d2
+            torch.cuda.empty_cache()
+        line["gpu_launches_all"] = (line["gpu_launches"] + line["prefill_fills_cache"]["gpu_launches"]
+                                    + line["prefill_via_cache"]["gpu_launches"]
+                                    + sum(line[n]["gpu_launches"] for n in EXTRA_PREFILL + EXTRA_DECODE))
 
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        if pre:
+    if with_cpu:
+        if args.workload and pre:
             v, desc, thr = oracle_prefill_sample(pre.spec, args.cpu_seconds)
             line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": thr,
                                     "kind": "oracle", "sample": desc}
-        else:
-            v, desc, thr = oracle_decode_sample(dec.spec, args.cpu_seconds)
+        elif args.workload:
+            if dec.spec.L_min >= (1 << 16):
+                v, desc, thr = oracle_decode_long_sample(dec)
+            else:
+                v, desc, thr = oracle_decode_sample(dec.spec, args.cpu_seconds)
             line["cpu_baseline"] = {"value": v, "unit": "GB/s", "cores": thr,
+                                    "kind": "oracle", "sample": desc}
+        else:
+            v, desc, thr = oracle_prefill_sample(WORKLOADS[DEFAULT_PREFILL], args.cpu_seconds)
+            line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": thr,
                                     "kind": "oracle", "sample": desc}
     if rank == 0:
         print(json.dumps(line), flush=True)

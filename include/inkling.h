@@ -35,6 +35,15 @@
  *  - `status` (optional, nullable, device int32): kernels OR error bits into it
  *    (INKLING_STATUS_* below) instead of trapping; the caller zeroes it and
  *    reads it after synchronising.
+ *  - Failures found on the device cannot be return codes: the calls return
+ *    before their kernels run.  A kernel that meets one reports it through
+ *    `status`, and every output row it could not compute (a bounded wait that
+ *    gave up, a decode sequence length outside [1, max_blocks*128]) is
+ *    written as NaN, in `out` and `lse` alike, so a caller that passes
+ *    status = NULL still cannot mistake it for a result.  A block-table
+ *    entry outside [0, num_blocks) is reported only through `status`: a
+ *    kernel reads block 0 in its place (the rows are finite but wrong) and
+ *    skips a write to it.
  */
 #ifndef INKLING_H
 #define INKLING_H
@@ -198,6 +207,56 @@ typedef struct {
 inkling_status inkling_sconv_out(const inkling_sconv_out_params *p, inkling_stream_t stream);
 
 /* --------------------------------------------------------------------------
+ * inkling_sconv_out_sharded — the output sconv sharded over channels across
+ * n_ranks tensor-parallel ranks, fused with its reduce-scatter and
+ * all-gather (vLLM Recipes "thinkingmachines/Inkling": Overview, "Short
+ * convolution", which shards the sconv across the channel dimension with a
+ * reduce-scatter / all-gather so that its cache and compute are not
+ * replicated on every rank; Performance, "sconv-aware TP sharding", where
+ * each rank stores only its channel shard of the sconv cache).
+ *
+ * Each rank holds a partial sum x_r [B, T, C] of the sconv's input (the
+ * output of a row-parallel projection).  The call made on rank `rank`
+ * computes the channels c in [rank*Cs, (rank+1)*Cs), Cs = C / n_ranks:
+ *   s[b,t,c] = bf16( x_0[b,t,c] + x_1[b,t,c] + ... )   (fp32, rank order)
+ *   y[b,t,c] = sum_{k=0..3} w[c,k] * s[b,t-k,c]        (as inkling_sconv_out)
+ * and stores y[:, :, shard] into the output buffer of EVERY rank, so that
+ * after all ranks' calls each y_r holds the full y.  The 3 rows of s before
+ * t = 0 come from `state`, this rank's shard [B, 3, Cs] of the sconv state
+ * (or zero when NULL), which is then updated in place to the last 3 rows of
+ * (old state, s).
+ *
+ * Pointers: x_parts and y_parts are HOST arrays of n_ranks device pointers.
+ * Every one of them must be readable / writable from the current device:
+ * this GPU's own memory, or a peer's memory mapped into this process (CUDA
+ * IPC, symmetric memory, or peer access).  The kernel reads and writes them
+ * with plain 16-byte loads and stores (no TMA, no multicast).  The arrays
+ * themselves are copied at the call and may be freed after it returns.
+ * Ordering is the caller's: every x_r must be complete before any rank's call
+ * starts, and a rank may read its y only after every rank's call has ended
+ * (e.g. a cross-rank barrier before and after).  No x_r may overlap any y_r.
+ * Errors: n_ranks outside [1, INKLING_SHARD_MAX_RANKS], rank outside
+ * [0, n_ranks), C not a positive multiple of 8 * n_ranks, or a NULL pointer:
+ * INKLING_ERR_INVALID, nothing launched.
+ * -------------------------------------------------------------------------- */
+#define INKLING_SHARD_MAX_RANKS 8
+
+typedef struct {
+    const void *const *x_parts; /* host [n_ranks]: device [B, T, C] bf16 partial sums */
+    void *const *y_parts;       /* host [n_ranks]: device [B, T, C] bf16 outputs */
+    const float *w;             /* device [C, 4] fp32 taps of all channels (tap 0 = current) */
+    void *state;                /* device [B, 3, C/n_ranks] bf16 state shard, or NULL */
+    int32_t n_ranks;            /* 1 .. INKLING_SHARD_MAX_RANKS */
+    int32_t rank;               /* the channel shard this call computes, 0 .. n_ranks-1 */
+    int32_t batch;              /* B >= 0 */
+    int32_t seq_len;            /* T >= 0 */
+    int32_t channels;           /* C, a positive multiple of 8 * n_ranks */
+} inkling_sconv_out_sharded_params;
+
+inkling_status inkling_sconv_out_sharded(const inkling_sconv_out_sharded_params *p,
+                                         inkling_stream_t stream);
+
+/* --------------------------------------------------------------------------
  * inkling_attn_prefill_paged — chunked prefill over the paged cache.
  *
  * A chunk of new tokens per sequence (variable lengths, rows packed): the
@@ -322,13 +381,19 @@ inkling_status inkling_attn_decode(const inkling_decode_params *p, void *workspa
  * that loads it, until the process exits; no allocation routine is called.
  *  - The first call on a device asks the runtime for that array's address on
  *    the current device; make that first call before any stream capture.
+ *    The address is kept with the id of the CUDA context it belongs to and is
+ *    asked for again when another context is current (after cudaDeviceReset,
+ *    or under a context the caller created), so such a call is again a
+ *    first call.
  *  - With num_splits = 0 the split count is lowered, if needed, until the
  *    partials fit (one split needs none).  An explicit num_splits whose
  *    partials exceed 8 MiB returns INKLING_ERR_INVALID and launches nothing.
  *  - All calls share the array and it keeps the last call's contents.  Every
- *    partial a call reads is written earlier by the same call, so nothing
- *    needs clearing, but calls that overlap on the GPU (e.g. on two streams
- *    at once, on one device) race with each other: serialise them.
+ *    partial a call reads is written earlier by the same call (a split that
+ *    cannot compute its rows writes a NaN partial, never leaves the slot
+ *    alone), so nothing needs clearing, but calls that overlap on the GPU
+ *    (e.g. on two streams at once, on one device) race with each other:
+ *    serialise them.
  * -------------------------------------------------------------------------- */
 inkling_status inkling_attn_decode_static(const inkling_decode_params *p, inkling_stream_t stream);
 

@@ -28,6 +28,7 @@ EXPORTED = (
     "inkling_selftest_wait_timeout",
     "inkling_sconv_kv",
     "inkling_sconv_out",
+    "inkling_sconv_out_sharded",
     "inkling_attn_prefill",
     "inkling_attn_prefill_paged",
     "inkling_attn_decode_workspace_bytes",
@@ -57,6 +58,15 @@ class PrefillParams(ctypes.Structure):
 
 class SconvOutParams(ctypes.Structure):
     _fields_ = [("x", _P), ("w", _P), ("state", _P), ("y", _P), ("batch", _I), ("seq_len", _I),
+                ("channels", _I)]
+
+
+SHARD_MAX_RANKS = 8
+
+
+class SconvOutShardedParams(ctypes.Structure):
+    _fields_ = [("x_parts", ctypes.POINTER(_P)), ("y_parts", ctypes.POINTER(_P)), ("w", _P),
+                ("state", _P), ("n_ranks", _I), ("rank", _I), ("batch", _I), ("seq_len", _I),
                 ("channels", _I)]
 
 
@@ -105,6 +115,8 @@ def load_library(path: str = LIB_PATH):
         lib.inkling_attn_prefill.restype = ctypes.c_int
         lib.inkling_sconv_out.argtypes = [ctypes.POINTER(SconvOutParams), _P]
         lib.inkling_sconv_out.restype = ctypes.c_int
+        lib.inkling_sconv_out_sharded.argtypes = [ctypes.POINTER(SconvOutShardedParams), _P]
+        lib.inkling_sconv_out_sharded.restype = ctypes.c_int
         lib.inkling_attn_prefill_paged.argtypes = [ctypes.POINTER(PrefillPagedParams), _P]
         lib.inkling_attn_prefill_paged.restype = ctypes.c_int
         lib.inkling_attn_decode_workspace_bytes.argtypes = [_I, _I, _I]
@@ -255,6 +267,37 @@ def sconv_out(x, w, state=None, out=None, stream=None):
     p = SconvOutParams(_ptr(x), _ptr(w), _ptr(state), _ptr(out), B, T, C)
     _check(load_library().inkling_sconv_out(ctypes.byref(p), _stream(stream)))
     return out
+
+
+def sconv_out_sharded(x_parts, w, y_parts, rank, state=None, stream=None):
+    """One rank's call of the output sconv sharded over channels, fused with
+    its reduce-scatter and all-gather (see inkling.h).  ``x_parts`` /
+    ``y_parts``: one [B, T, C] bf16 tensor per rank (the partial sums and the
+    outputs), each readable / writable from this device; ``state``: this
+    rank's [B, 3, C / n] shard of the sconv state or None.  Writes channels
+    [rank * C/n, (rank+1) * C/n) of the sconv of the summed input into every
+    y_parts[r]; the caller orders the ranks' calls (inputs complete before,
+    outputs read after every rank's call)."""
+    n = len(x_parts)
+    if n < 1 or n > SHARD_MAX_RANKS or len(y_parts) != n:
+        raise ValueError(f"x_parts and y_parts must hold the same 1..{SHARD_MAX_RANKS} tensors")
+    B, T, C = x_parts[0].shape
+    for i, t in enumerate(list(x_parts) + list(y_parts)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or tuple(t.shape) != (B, T, C):
+            raise ValueError(f"part {i} must be a bf16 [B, T, C] tensor like x_parts[0]")
+        if not t.is_contiguous():
+            raise ValueError(f"part {i} must be contiguous")
+    _dev(w, torch.float32, "w", 2)
+    if w.shape != (C, 4):
+        raise ValueError("w must be [C, 4]")
+    if state is not None:
+        _dev(state, torch.bfloat16, "state", 3)
+        if tuple(state.shape) != (B, 3, C // n):
+            raise ValueError("state must be [B, 3, C / n_ranks]")
+    xs = (_P * n)(*[t.data_ptr() for t in x_parts])
+    ys = (_P * n)(*[t.data_ptr() for t in y_parts])
+    p = SconvOutShardedParams(xs, ys, _ptr(w), _ptr(state), n, int(rank), B, T, C)
+    _check(load_library().inkling_sconv_out_sharded(ctypes.byref(p), _stream(stream)))
 
 
 def attn_prefill_paged(q, cu_q, k_cache, v_cache, block_table, seq_lens, bias, window=0,

@@ -17,7 +17,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libinkling.so")
 SOURCES = ["api.cu", "sconv_kv.cu", "attn_decode.cu", "attn_prefill.cu", "attn_prefill_pair.cu",
-           "attn_prefill_paged.cu", "sconv_out.cu", "attn_decode_mq.cu"]
+           "attn_prefill_paged.cu", "sconv_out.cu", "attn_decode_mq.cu", "sconv_shard.cu"]
 HEADERS = ["common.cuh", "prefill_common.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

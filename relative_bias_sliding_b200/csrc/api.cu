@@ -13,6 +13,8 @@ cudaError_t launch_sconv_kv(const inkling_sconv_params &p, cudaStream_t stream);
 cudaError_t launch_attn_prefill(const inkling_prefill_params &p, const CUtensorMap *maps,
                                 cudaStream_t stream);
 cudaError_t launch_sconv_out(const inkling_sconv_out_params &p, cudaStream_t stream);
+cudaError_t launch_sconv_out_sharded(const inkling_sconv_out_sharded_params &p,
+                                     cudaStream_t stream);
 cudaError_t launch_attn_decode_mq(const inkling_decode_params &p, int splits, void *workspace,
                                   const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                                   const CUtensorMap &tm_v, cudaStream_t stream);
@@ -326,6 +328,44 @@ inkling_status inkling_sconv_out(const inkling_sconv_out_params *p, inkling_stre
     return INKLING_OK;
 }
 
+inkling_status inkling_sconv_out_sharded(const inkling_sconv_out_sharded_params *p,
+                                         inkling_stream_t stream) {
+    g_err[0] = 0;
+    if (!p) return fail(INKLING_ERR_INVALID, "params is NULL");
+    if (p->n_ranks < 1 || p->n_ranks > INKLING_SHARD_MAX_RANKS)
+        return fail(INKLING_ERR_INVALID, "n_ranks must be in [1, %d]", INKLING_SHARD_MAX_RANKS);
+    if (p->rank < 0 || p->rank >= p->n_ranks)
+        return fail(INKLING_ERR_INVALID, "rank must be in [0, n_ranks)");
+    if (p->batch < 0 || p->seq_len < 0) return fail(INKLING_ERR_INVALID, "batch and seq_len must be >= 0");
+    if (p->channels < 8 * p->n_ranks || p->channels % (8 * p->n_ranks))
+        return fail(INKLING_ERR_INVALID, "channels must be a positive multiple of 8 * n_ranks");
+    if ((long)p->batch * p->seq_len * p->channels >= (1L << 40))
+        return fail(INKLING_ERR_UNSUPPORTED, "tensor too large");
+    if (p->batch == 0 || p->seq_len == 0) return INKLING_OK;
+    if (!p->x_parts || !p->y_parts || !p->w)
+        return fail(INKLING_ERR_INVALID, "x_parts, y_parts and w must not be NULL");
+    if (!aligned16(p->w) || (p->state && !aligned16(p->state)))
+        return fail(INKLING_ERR_INVALID, "w and state must be 16-byte aligned");
+    const size_t nb = (size_t)p->batch * p->seq_len * p->channels * 2;
+    for (int r = 0; r < p->n_ranks; ++r) {
+        if (!p->x_parts[r] || !p->y_parts[r])
+            return fail(INKLING_ERR_INVALID, "x_parts[%d] / y_parts[%d] is NULL", r, r);
+        if (!aligned16(p->x_parts[r]) || !aligned16(p->y_parts[r]))
+            return fail(INKLING_ERR_INVALID, "x_parts and y_parts must be 16-byte aligned");
+    }
+    for (int r = 0; r < p->n_ranks; ++r)
+        for (int q = 0; q < p->n_ranks; ++q) {
+            const char *x0 = (const char *)p->x_parts[r], *y0 = (const char *)p->y_parts[q];
+            if (x0 < y0 + nb && y0 < x0 + nb)
+                return fail(INKLING_ERR_INVALID, "x_parts[%d] overlaps y_parts[%d]", r, q);
+        }
+    inkling_status st = check_device(nullptr);
+    if (st != INKLING_OK) return st;
+    cudaError_t e = launch_sconv_out_sharded(*p, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "sconv_out_sharded launch");
+    return INKLING_OK;
+}
+
 inkling_status inkling_attn_prefill_paged(const inkling_prefill_paged_params *p,
                                           inkling_stream_t stream) {
     g_err[0] = 0;
@@ -437,6 +477,11 @@ inkling_status inkling_attn_decode_static(const inkling_decode_params *p, inklin
 static inkling_status decode_with(const inkling_decode_params *p, int splits, void *workspace,
                                   size_t workspace_bytes, inkling_stream_t stream) {
     inkling_status st;
+    // one thread block per (sequence, kv head, split): the grid must fit a
+    // signed 32-bit count
+    if ((long)p->num_seqs * p->num_kv_heads * splits >= (1L << 31))
+        return fail(INKLING_ERR_UNSUPPORTED, "num_seqs * num_kv_heads * splits (%d) exceeds 2^31",
+                    splits);
     if (splits > 1) {
         const size_t need = inkling_attn_decode_workspace_bytes(decode_rows(*p), p->num_q_heads, splits);
         if (!workspace || workspace_bytes < need)

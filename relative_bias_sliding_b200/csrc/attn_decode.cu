@@ -78,6 +78,9 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
     const int s = blockIdx.x % a.S;
     const int kvh = (blockIdx.x / a.S) % a.Hkv;
     const int split = blockIdx.x / (a.S * a.Hkv);
+    // the combine kernel that follows (with splits) may launch now; it waits
+    // for this whole grid before reading a partial
+    if (a.splits > 1) pdl_launch_dependents();
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kDecStages; ++i) {
@@ -267,7 +270,23 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
         named_bar_sync(1, 128);
         const int u = threadIdx.x;  // 0..127
         const int gg = u >> 4, d0 = (u & 15) * 8;
-        if (gg < a.G && !*abort_flag) {
+        if (gg < a.G && (bad_len || *abort_flag)) {
+            // a row this call could not compute (its length is out of range, or
+            // a bounded wait gave up) reads NaN, so that a caller without a
+            // status word cannot take it, or another call's partial, for a
+            // result; with splits the NaN partial makes the merged row NaN
+            const float nanv = __int_as_float(0x7fc00000);
+            const int hh = kvh * a.G + gg;
+            if (a.splits == 1) {
+                const uint32_t nb = 0x7fc07fc0u;
+                *(uint4 *)(a.out + ((long)s * a.Hq + hh) * 128 + d0) = make_uint4(nb, nb, nb, nb);
+                if (a.lse && (u & 15) == 0) a.lse[(long)s * a.Hq + hh] = nanv;
+            } else if ((u & 15) == 0) {
+                const long pi = ((long)s * a.Hq + hh) * a.splits + split;
+                a.part_ml[pi * 2] = nanv;
+                a.part_ml[pi * 2 + 1] = nanv;
+            }
+        } else if (gg < a.G) {
             float M = -INFINITY;
 #pragma unroll
             for (int w = 0; w < 4; ++w) M = fmaxf(M, red_ml[(w * 8 + gg) * 2]);
@@ -319,6 +338,9 @@ decode_combine_kernel(const float *__restrict__ part_o, const float *__restrict_
                       uint16_t *__restrict__ out, float *__restrict__ lse, int pairs, int splits) {
     const int pair = blockIdx.x * 4 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
+    // launched programmatically behind the split kernel: its partials are
+    // complete and visible only after this wait
+    pdl_wait_primary();
     if (pair >= pairs) return;
     const float *ml = part_ml + (long)pair * splits * 2;
     float M = -INFINITY;
@@ -339,19 +361,36 @@ decode_combine_kernel(const float *__restrict__ part_o, const float *__restrict_
         acc.z = fmaf(f, v.z, acc.z);
         acc.w = fmaf(f, v.w, acc.w);
     }
+    // a NaN partial (a split that could not compute its rows) makes Ls, the
+    // output and the lse NaN
     const float inv = (Ls > 0.f) ? 1.f / Ls : 0.f;
     uint2 pk;
     pk.x = pack_bf16(acc.x * inv, acc.y * inv);
     pk.y = pack_bf16(acc.z * inv, acc.w * inv);
     *(uint2 *)(out + (long)pair * 128 + lane * 4) = pk;
     if (lse && lane == 0)
-        lse[pair] = (Ls > 0.f) ? (M + __log2f(Ls)) * 0.6931471805599453f : -INFINITY;
+        lse[pair] = (Ls > 0.f) ? (M + __log2f(Ls)) * 0.6931471805599453f
+                               : (Ls == 0.f ? -INFINITY : Ls);
 }
 
+// The combine is launched with programmatic dependent launch: its launch
+// overlaps the tail of the split kernel, which lets it start at its first
+// block, and its blocks wait for the split kernel's partials on the device.
 cudaError_t launch_decode_combine(const float *part_o, const float *part_ml, uint16_t *out, float *lse,
                                   long rows, int splits, cudaStream_t stream) {
-    decode_combine_kernel<<<(unsigned)((rows + 3) / 4), 128, 0, stream>>>(part_o, part_ml, out, lse,
-                                                                        (int)rows, splits);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((rows + 3) / 4), 1, 1);
+    cfg.blockDim = dim3(128, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, decode_combine_kernel, part_o, part_ml, out, lse,
+                                       (int)rows, splits);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -386,9 +425,7 @@ cudaError_t launch_attn_decode(const inkling_decode_params &p, int splits, void 
     decode_split_kernel<<<(unsigned)grid, 160, kDecSmem, stream>>>(tm_k, tm_v, a);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || splits == 1) return e;
-    decode_combine_kernel<<<(unsigned)((rows_total + 3) / 4), 128, 0, stream>>>(
-        a.part_o, a.part_ml, a.out, a.lse, (int)rows_total, splits);
-    return cudaGetLastError();
+    return launch_decode_combine(a.part_o, a.part_ml, a.out, a.lse, rows_total, splits, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -396,26 +433,64 @@ cudaError_t launch_attn_decode(const inkling_decode_params &p, int splits, void 
 // allocate device memory themselves (see inkling_attn_decode_static).  The
 // array is part of this module: every device that loads the library holds
 // kDecodeStaticScratchBytes of it until the process exits.  Host code never
-// dereferences the symbol; it asks the runtime for the device address once
-// per device (with that device current) and hands that address to the kernels.
+// dereferences the symbol; it asks the runtime for the device address (with
+// that device current) and hands that address to the kernels.  The address
+// is kept per device together with the unique id of the CUDA context it was
+// resolved in, and resolved again when the current context is another one
+// (after cudaDeviceReset, or under a context the caller made current).
 constexpr size_t kDecodeStaticScratchBytes = (size_t)8 << 20;
 static __device__ __align__(256) unsigned char g_decode_scratch[kDecodeStaticScratchBytes];
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+
+// unique id of the current CUDA context; false when no context is current or
+// the driver does not provide the entry points
+static bool current_context_id(unsigned long long *id) {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = (CtxGetCurrentFn)p;
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = (CtxGetIdFn)p;
+    });
+    if (!get_current || !get_id) return false;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
 
 cudaError_t decode_static_scratch(void **ptr, size_t *bytes) {
     static std::mutex mu;
     static void *addr[64] = {nullptr};
+    static unsigned long long ctx_of[64] = {0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    unsigned long long id = 0;
+    bool have_id = current_context_id(&id);
     std::lock_guard<std::mutex> lock(mu);
-    if (addr[dev] == nullptr) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_decode_scratch);
-        if (e != cudaSuccess) return e;
-        addr[dev] = p;
+    if (have_id && addr[dev] != nullptr && ctx_of[dev] == id) {
+        *ptr = addr[dev];
+        *bytes = kDecodeStaticScratchBytes;
+        return cudaSuccess;
     }
-    *ptr = addr[dev];
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess) return e;
+    // the runtime has made its context current if none was
+    if (!have_id) have_id = current_context_id(&id);
+    addr[dev] = have_id ? p : nullptr;  // without an id, resolve on every call
+    ctx_of[dev] = id;
+    *ptr = p;
     *bytes = kDecodeStaticScratchBytes;
     return cudaSuccess;
 }

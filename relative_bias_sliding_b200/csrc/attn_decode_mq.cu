@@ -83,6 +83,9 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int kvh = (blockIdx.x / a.S) % a.Hkv;
     const int split = blockIdx.x / (a.S * a.Hkv);
     const int Q = a.Q, G = a.G, rows = G * Q;
+    // the combine kernel that follows (with splits) may launch now; it waits
+    // for this whole grid before reading a partial
+    if (a.splits > 1) pdl_launch_dependents();
 
     // key tiles of this sequence (union of its rows' windows) and this split
     const int L = a.seq_lens[s];
@@ -295,7 +298,24 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tmem_wait_ld();
         }
         auto o = [&](int i) { return __uint_as_float(ob[i]); };
-        if (rv && !bad_len && !*abort_flag) {
+        if (rv && (bad_len || *abort_flag)) {
+            // a row this call could not compute (length out of range, or a
+            // bounded wait gave up) reads NaN; with splits, a NaN partial
+            // makes the merged row NaN
+            const long pair = ((long)s * Q + qi) * a.Hq + h;
+            const float nanv = __int_as_float(0x7fc00000);
+            if (a.splits == 1) {
+                const uint32_t nb = 0x7fc07fc0u;
+                uint4 *dst = (uint4 *)(a.out + pair * 128);
+#pragma unroll
+                for (int c = 0; c < 16; ++c) dst[c] = make_uint4(nb, nb, nb, nb);
+                if (a.lse) a.lse[pair] = nanv;
+            } else {
+                const long pi = pair * a.splits + split;
+                a.part_ml[pi * 2] = nanv;
+                a.part_ml[pi * 2 + 1] = nanv;
+            }
+        } else if (rv) {
             const long pair = ((long)s * Q + qi) * a.Hq + h;
             if (a.splits == 1) {
                 const float inv = (l > 0.f) ? 1.f / l : 0.f;

@@ -61,9 +61,18 @@ struct RowStoreEpilogue {
     int Hq, h;
     INK_DEV void operator()(bool have_o, int u, int, float l, float m_ref, uint32_t o_col,
                             volatile int *) const {
-        if (!have_o) return;  // warp-uniform: emit_row's TMEM loads need the whole warp
         const bool store = u < rows_valid;
         uint16_t *dst = out + ((row0 + u) * Hq + h) * 128;
+        if (!have_o) {
+            // a bounded wait gave up: the row reads NaN (the status word says why)
+            if (store) {
+                const uint32_t nb = 0x7fc07fc0u;
+#pragma unroll
+                for (int c = 0; c < 16; ++c) *(uint4 *)(dst + c * 8) = make_uint4(nb, nb, nb, nb);
+                if (lse) lse[(row0 + u) * Hq + h] = __int_as_float(0x7fc00000);
+            }
+            return;  // warp-uniform: emit_row's TMEM loads need the whole warp
+        }
         emit_row(o_col, l, [&](int c, uint4 v) {
             if (store) *(uint4 *)(dst + c * 8) = v;
         });

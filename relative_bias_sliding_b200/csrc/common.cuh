@@ -136,6 +136,23 @@ INK_DEV void tma_store_4d(const CUtensorMap *m, const void *src, int x, int y, i
 INK_DEV void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // wait until every committed bulk store of this thread has completed
 INK_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// wait until every committed bulk store of this thread has finished READING
+// its shared-memory source (the writes to global memory complete on their
+// own, before the grid completes): enough before the source is reused or the
+// block exits
+INK_DEV void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
+// Compiler-level fence on 32 registers written by an asynchronous tcgen05.ld:
+// placed after tcgen05.wait::ld, it keeps every use of them after the wait.
+INK_DEV void reg_fence32(uint32_t *r) {
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                   "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                   "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                   "+r"(r[30]), "+r"(r[31]));
+}
 
 // generic-proxy shared-memory writes -> visible to the async proxy (tensor core)
 INK_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
@@ -353,6 +370,15 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major, 
            ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) |
            ((uint32_t)(M >> 4) << 24);
 }
+
+// ------------------------------------------- programmatic dependent launch --
+// A kernel launched with the programmatic-stream-serialization attribute may
+// start while the kernel before it on the stream is still running; it waits
+// here until that kernel has completed and its memory operations are visible.
+INK_DEV void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the dependent kernel of the stream launch now (its blocks then wait in
+// pdl_wait_primary for this whole grid); issued by each block at its start.
+INK_DEV void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ------------------------------------------------------------- numerics --
 

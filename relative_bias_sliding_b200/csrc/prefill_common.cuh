@@ -195,6 +195,13 @@ struct TmaStoreEpilogue {
             if (a.lse && i < a.T)
                 a.lse[((long)b * a.Hq + h) * a.T + i] = (l > 0.f) ? m_ref + __logf(l) : -INFINITY;
             fence_proxy_async_smem();
+        } else if (i < a.T) {
+            // a bounded wait gave up: the row reads NaN (the status word says why)
+            const uint32_t nb = 0x7fc07fc0u;
+            uint16_t *dst = a.out + (((long)b * a.T + i) * a.Hq + h) * 128;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) *(uint4 *)(dst + c * 8) = make_uint4(nb, nb, nb, nb);
+            if (a.lse) a.lse[((long)b * a.Hq + h) * a.T + i] = __int_as_float(0x7fc00000);
         }
         // every warp of the group reaches this barrier (have_o is uniform per warp)
         named_bar_sync(bar_id, 128);
@@ -202,7 +209,7 @@ struct TmaStoreEpilogue {
             tma_store_4d(tm_out, stage, 0, r0, h, b);
             tma_store_4d(tm_out, stage + 16384, 64, r0, h, b);
             bulk_commit_group();
-            bulk_wait_all();
+            bulk_wait_read_all();
         }
     }
 };
@@ -259,12 +266,16 @@ INK_DEV void softmax_role(const PrefillArgs &a, float *bias_sm, uint64_t *s_full
         if (!dead) dead = !mbar_wait_warp(&s_full[t], k & 1, abort_flag, a.status);
         if (dead) continue;  // keep stepping through the group barrier
         tc_fence_after();
+        // S in two halves: the second half's load runs while the first
+        // half's logits are computed
         uint32_t sr[128];
         tmem_ld32(s_col + 0, sr + 0);
         tmem_ld32(s_col + 32, sr + 32);
+        tmem_wait_ld();
+        reg_fence32(sr + 0);
+        reg_fence32(sr + 32);
         tmem_ld32(s_col + 64, sr + 64);
         tmem_ld32(s_col + 96, sr + 96);
-        tmem_wait_ld();
         const float4 *rp = (const float4 *)(bb + sh * kBiasCopy + (o_rd - sh));
         float x[128];
         const int dist0 = i - j0;  // distance of key j0 + c is dist0 - c
@@ -283,9 +294,9 @@ INK_DEV void softmax_role(const PrefillArgs &a, float *bias_sm, uint64_t *s_full
 #pragma unroll
         for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
         const f32x2 sc2 = pk2(scale, scale);
-        auto logits = [&](auto masked) {
+        auto logits = [&](auto masked, auto half) {
 #pragma unroll
-            for (int cb = 0; cb < 4; ++cb) {
+            for (int cb = 2 * decltype(half)::value; cb < 2 * decltype(half)::value + 2; ++cb) {
                 float4 b4[8];
 #pragma unroll
                 for (int j = 0; j < 8; ++j) b4[j] = rp[cb * 8 + j];
@@ -307,10 +318,19 @@ INK_DEV void softmax_role(const PrefillArgs &a, float *bias_sm, uint64_t *s_full
                 }
             }
         };
+        using H0 = std::integral_constant<int, 0>;
+        using H1 = std::integral_constant<int, 1>;
         if (full)
-            logits(std::false_type{});
+            logits(std::false_type{}, H0{});
         else
-            logits(std::true_type{});
+            logits(std::true_type{}, H0{});
+        tmem_wait_ld();
+        reg_fence32(sr + 64);
+        reg_fence32(sr + 96);
+        if (full)
+            logits(std::false_type{}, H1{});
+        else
+            logits(std::true_type{}, H1{});
         const float mx =
             fmaxf(max3f(m8[0], m8[1], m8[2]), max3f(max3f(m8[3], m8[4], m8[5]), m8[6], m8[7]));
         // lazy rescale: move the reference only when the max grows by > tau
@@ -326,17 +346,21 @@ INK_DEV void softmax_role(const PrefillArgs &a, float *bias_sm, uint64_t *s_full
             const f32x2 l2e2 = pk2(kLog2e, kLog2e), mneg2 = pk2(mneg, mneg);
             f32x2 acc[4] = {0ull, 0ull, 0ull, 0ull};
             uint32_t pk[64];
+            // P in two halves of 64 keys: the first half's store to tensor
+            // memory runs while the second half's exponentials are computed
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                const f32x2 tt = ffma2(pk2(x[2 * c], x[2 * c + 1]), l2e2, mneg2);
-                float t0, t1;
-                upk2(tt, t0, t1);
-                const float p0 = ex2(t0), p1 = ex2(t1);
-                acc[c & 3] = fadd2(acc[c & 3], pk2(p0, p1));
-                pk[c] = pack_bf16(p0, p1);
+            for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+                for (int c = 32 * hf; c < 32 * hf + 32; ++c) {
+                    const f32x2 tt = ffma2(pk2(x[2 * c], x[2 * c + 1]), l2e2, mneg2);
+                    float t0, t1;
+                    upk2(tt, t0, t1);
+                    const float p0 = ex2(t0), p1 = ex2(t1);
+                    acc[c & 3] = fadd2(acc[c & 3], pk2(p0, p1));
+                    pk[c] = pack_bf16(p0, p1);
+                }
+                tmem_st32(s_col + 32 * hf, pk + 32 * hf);
             }
-            tmem_st32(s_col + 0, pk + 0);
-            tmem_st32(s_col + 32, pk + 32);
             const f32x2 s01 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
             float la, lb;
             upk2(s01, la, lb);

@@ -56,6 +56,9 @@ int main(void) {{
   F(inkling_prefill_paged_params, max_q) F(inkling_prefill_paged_params, d_max)
   printf("sconv_out %zu\\n", sizeof(inkling_sconv_out_params));
   F(inkling_sconv_out_params, y) F(inkling_sconv_out_params, channels)
+  printf("sharded %zu\\n", sizeof(inkling_sconv_out_sharded_params));
+  F(inkling_sconv_out_sharded_params, state) F(inkling_sconv_out_sharded_params, n_ranks)
+  F(inkling_sconv_out_sharded_params, channels)
   return 0;
 }}""")
     exe = tmp_path / "sizes"
@@ -81,6 +84,31 @@ int main(void) {{
     assert int(out["sconv_out"]) == ctypes.sizeof(O)
     assert int(out["inkling_sconv_out_params y"]) == O.y.offset
     assert int(out["inkling_sconv_out_params channels"]) == O.channels.offset
+    H = binding.SconvOutShardedParams
+    assert int(out["sharded"]) == ctypes.sizeof(H)
+    for m in ("state", "n_ranks", "channels"):
+        assert int(out["inkling_sconv_out_sharded_params " + m]) == getattr(H, m).offset
+
+
+def test_sharded_sconv_validation_rejects_before_launch(lib):
+    # argument checks come before any device access (addresses never read)
+    f = lib.inkling_sconv_out_sharded
+    fake = [ctypes.c_void_p((1 << 20) + (i << 24)) for i in range(4)]
+    xs = (ctypes.c_void_p * 2)(fake[0], fake[1])
+    ys = (ctypes.c_void_p * 2)(fake[2], fake[3])
+    p = binding.SconvOutShardedParams(xs, ys, fake[0], None, 2, 0, 1, 16, 256)
+    p.n_ranks = 9
+    assert f(ctypes.byref(p), None) == binding.INKLING_ERR_INVALID
+    p.n_ranks, p.rank = 2, 2
+    assert f(ctypes.byref(p), None) == binding.INKLING_ERR_INVALID
+    p.rank, p.channels = 1, 24   # not a multiple of 8 * n_ranks
+    assert f(ctypes.byref(p), None) == binding.INKLING_ERR_INVALID
+    p.channels = 256
+    p.y_parts = (ctypes.c_void_p * 2)(fake[2], fake[1])   # y_parts[1] is x_parts[1]
+    assert f(ctypes.byref(p), None) == binding.INKLING_ERR_INVALID
+    assert b"overlaps" in lib.inkling_last_error()
+    p.seq_len = 0
+    assert f(ctypes.byref(p), None) == binding.INKLING_OK   # empty: no-op
 
 
 def test_workspace_bytes(lib):

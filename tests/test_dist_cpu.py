@@ -59,3 +59,79 @@ def test_single_rank_has_no_process_group():
     import bench
     assert bench.init_dist(1, "gloo") is None
     assert bench.max_over_ranks(None, [3.0, 1.0]) == [3.0, 1.0]
+
+
+def _bits(t):
+    import torch
+    return t.contiguous().view(torch.int16).numpy().view("uint16")
+
+
+def _oracle_sconv_inplace(xs, w_shard, state_shard):
+    """The oracle's sconv standing in, on the CPU, for the library's kernel in
+    the channel-sharded output sconv (test infrastructure: only the collective
+    logic around it is under test here).  Updates state_shard in place."""
+    import numpy as np
+    import torch
+    import oracle
+    y = oracle.sconv(_bits(xs), w_shard.numpy(), None if state_shard is None else _bits(state_shard))
+    if state_shard is not None:
+        hist = torch.cat([state_shard, xs], dim=1)
+        state_shard.copy_(hist[:, -3:])
+    return torch.from_numpy(np.ascontiguousarray(y).view(np.int16)).view(torch.bfloat16)
+
+
+def _sconv_worker(rank, world, port, q):
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import torch
+    import torch.distributed as dist
+    from relative_bias_sliding_b200.sharded import channel_shard, sconv_out_reduce_scatter
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    B, T, C = 2, 70, 64
+    g = torch.Generator().manual_seed(100)  # the same draws on every rank
+    xs = [torch.randn(B, T, C, generator=g).to(torch.bfloat16) for _ in range(world)]
+    w = torch.randn(C, 4, generator=g) * 0.5
+    state = torch.randn(B, 3, C, generator=g).to(torch.bfloat16)
+    sl = channel_shard(C, world, rank)
+    st = state[:, :, sl].clone()
+    y = sconv_out_reduce_scatter(xs[rank], w, st, local_sconv=_oracle_sconv_inplace)
+    y2 = sconv_out_reduce_scatter(xs[rank], w, st, local_sconv=_oracle_sconv_inplace)
+    dist.destroy_process_group()
+    q.put((rank, _bits(y).copy(), _bits(y2).copy(), _bits(st).copy()))
+
+
+def test_channel_sharded_output_sconv_gloo_world2():
+    """Two ranks each hold a partial sum of the output sconv's input; the
+    reduce-scatter / sconv-of-the-shard / all-gather path returns on every
+    rank the unsharded sconv of the summed input, bit for bit, twice in a row
+    (the second call continues from the state shards), and each rank's state
+    shard equals its slice of the unsharded state."""
+    import torch
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    world = 2
+    procs = [ctx.Process(target=_sconv_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = {r: (y, y2, st) for r, y, y2, st in (q.get(timeout=120) for _ in procs)}
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    # unsharded reference on one process: sum in fp32, one bf16 rounding,
+    # sconv of all channels from the full state, twice
+    sys.path.insert(0, ROOT)
+    from relative_bias_sliding_b200.sharded import channel_shard
+    B, T, C = 2, 70, 64
+    g = torch.Generator().manual_seed(100)
+    xs = [torch.randn(B, T, C, generator=g).to(torch.bfloat16) for _ in range(world)]
+    w = torch.randn(C, 4, generator=g) * 0.5
+    state = torch.randn(B, 3, C, generator=g).to(torch.bfloat16)
+    s = (xs[0].float() + xs[1].float()).to(torch.bfloat16)
+    y_ref = _oracle_sconv_inplace(s, w, state)
+    y2_ref = _oracle_sconv_inplace(s, w, state)
+    for r in range(world):
+        y, y2, st = out[r]
+        assert (y == _bits(y_ref)).all(), f"rank {r}: first call"
+        assert (y2 == _bits(y2_ref)).all(), f"rank {r}: second call"
+        assert (st == _bits(state[:, :, channel_shard(C, world, r)])).all(), f"rank {r}: state"
