@@ -124,7 +124,7 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (ok[t])
             softmax_role(a, (float *)(smem + SM_BIAS) + t * 2 * kBiasBuf, &bar[B_SFULL],
                          &bar[B_ODONE], abort_flag, tbase, t, h, r0[t], a.T, lo[t], hi[t], 3 + t,
-                         [&](int tt) { mbar_arrive(&bar[B_PFULL + tt]); },
+                         0, 0u, [&](int tt) { mbar_arrive(&bar[B_PFULL + tt]); },
                          TmaStoreEpilogue{a, smem + SM_Q + t * 32768, &tm_out, b, h, r0[t], 3 + t});
     } else if (warp < 12) {
         // ========================== sconv transform: warps 8-9 keys, 10-11 values ==

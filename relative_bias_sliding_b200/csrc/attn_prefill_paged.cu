@@ -152,7 +152,7 @@ attn_prefill_paged_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (ok[t])
             softmax_role(a, (float *)(smem + PG_BIAS) + t * 2 * kBiasBuf, &bar[G_SFULL],
                          &bar[G_ODONE], abort_flag, tbase, t, h, base + r0[t], L, lo[t], hi[t],
-                         3 + t, [&](int tt) { mbar_arrive(&bar[G_PFULL + tt]); },
+                         3 + t, 0, 0u, [&](int tt) { mbar_arrive(&bar[G_PFULL + tt]); },
                          RowStoreEpilogue{g.out, g.lse, (long)q_begin + r0[t], n - r0[t], a.Hq, h});
     } else if (warp < 12) {
         setmaxnreg_dec80();

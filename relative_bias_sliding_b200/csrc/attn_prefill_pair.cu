@@ -167,7 +167,7 @@ attn_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int t = warp >> 2;
         if (ok[t])
             softmax_role(a, (float *)(smem + PBIAS) + t * 2 * kBiasBuf, &bar[S_FULL], &bar[O_DONE],
-                         abort_flag, tbase, t, hd[t], r0[t], a.T, lo[t], hi[t], 3 + t,
+                         abort_flag, tbase, t, hd[t], r0[t], a.T, lo[t], hi[t], 3 + t, 0, 0u,
                          [&](int tt) {
                              __syncwarp();
                              if (lane == 0) mbar_arrive_cta_relaxed(&bar[P_FULL + tt], 0);

@@ -142,18 +142,6 @@ INK_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "m
 // block exits
 INK_DEV void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
-// Compiler-level fence on 32 registers written by an asynchronous tcgen05.ld:
-// placed after tcgen05.wait::ld, it keeps every use of them after the wait.
-INK_DEV void reg_fence32(uint32_t *r) {
-    asm volatile(""
-                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
-                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
-                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
-                   "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
-                   "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
-                   "+r"(r[30]), "+r"(r[31]));
-}
-
 // generic-proxy shared-memory writes -> visible to the async proxy (tensor core)
 INK_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 

@@ -224,11 +224,14 @@ struct TmaStoreEpilogue {
 // tile's two bias-diagonal buffers; `bar_id` is a named barrier private to
 // this warpgroup.  At the end every thread calls
 // epilogue(have_o, u, pos0 + u, l, m_ref, o_col, abort_flag).
+// `k_base` counts the key tiles this group processed before (for the parities
+// of S_FULL and of the bias buffers when the group walks several work items),
+// `o_phase` is the parity of this item's O_DONE phase.
 template <class SignalP, class Epilogue>
 INK_DEV void softmax_role(const PrefillArgs &a, float *bias_sm, uint64_t *s_full, uint64_t *o_done,
                           volatile int *abort_flag, uint32_t tbase, int t, int h, int pos0,
-                          int key_end, int lo, int hi, int bar_id, SignalP signal_p,
-                          const Epilogue &epilogue) {
+                          int key_end, int lo, int hi, int bar_id, int k_base, uint32_t o_phase,
+                          SignalP signal_p, const Epilogue &epilogue) {
     const int u = threadIdx.x & 127;
     const uint32_t tl = tbase + ((uint32_t)(((threadIdx.x >> 5) & 3) * 32) << 16);
     const uint32_t s_col = tl + t * 128, o_col = tl + 256 + t * 128;
@@ -248,7 +251,8 @@ INK_DEV void softmax_role(const PrefillArgs &a, float *bias_sm, uint64_t *s_full
         // R[q] = bias[h, clamp(top - q, 0, d_max)], q = 0..254, top = pos0 - j0 + 127,
         // as 4 copies shifted by 0..3 floats so that row u reads R[127-u+c],
         // c = 0..127, with aligned 16-byte loads.  Double-buffered by tile parity.
-        float *bb = bias_sm + (k & 1) * kBiasBuf;
+        const int kk = k_base + k;
+        float *bb = bias_sm + (kk & 1) * kBiasBuf;
         {
             const int top = pos0 - j0 + 127;
 #pragma unroll
@@ -263,19 +267,15 @@ INK_DEV void softmax_role(const PrefillArgs &a, float *bias_sm, uint64_t *s_full
             }
         }
         named_bar_sync(bar_id, 128);
-        if (!dead) dead = !mbar_wait_warp(&s_full[t], k & 1, abort_flag, a.status);
+        if (!dead) dead = !mbar_wait_warp(&s_full[t], kk & 1, abort_flag, a.status);
         if (dead) continue;  // keep stepping through the group barrier
         tc_fence_after();
-        // S in two halves: the second half's load runs while the first
-        // half's logits are computed
         uint32_t sr[128];
         tmem_ld32(s_col + 0, sr + 0);
         tmem_ld32(s_col + 32, sr + 32);
-        tmem_wait_ld();
-        reg_fence32(sr + 0);
-        reg_fence32(sr + 32);
         tmem_ld32(s_col + 64, sr + 64);
         tmem_ld32(s_col + 96, sr + 96);
+        tmem_wait_ld();
         const float4 *rp = (const float4 *)(bb + sh * kBiasCopy + (o_rd - sh));
         float x[128];
         const int dist0 = i - j0;  // distance of key j0 + c is dist0 - c
@@ -294,9 +294,9 @@ INK_DEV void softmax_role(const PrefillArgs &a, float *bias_sm, uint64_t *s_full
 #pragma unroll
         for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
         const f32x2 sc2 = pk2(scale, scale);
-        auto logits = [&](auto masked, auto half) {
+        auto logits = [&](auto masked) {
 #pragma unroll
-            for (int cb = 2 * decltype(half)::value; cb < 2 * decltype(half)::value + 2; ++cb) {
+            for (int cb = 0; cb < 4; ++cb) {
                 float4 b4[8];
 #pragma unroll
                 for (int j = 0; j < 8; ++j) b4[j] = rp[cb * 8 + j];
@@ -318,19 +318,10 @@ INK_DEV void softmax_role(const PrefillArgs &a, float *bias_sm, uint64_t *s_full
                 }
             }
         };
-        using H0 = std::integral_constant<int, 0>;
-        using H1 = std::integral_constant<int, 1>;
         if (full)
-            logits(std::false_type{}, H0{});
+            logits(std::false_type{});
         else
-            logits(std::true_type{}, H0{});
-        tmem_wait_ld();
-        reg_fence32(sr + 64);
-        reg_fence32(sr + 96);
-        if (full)
-            logits(std::false_type{}, H1{});
-        else
-            logits(std::true_type{}, H1{});
+            logits(std::true_type{});
         const float mx =
             fmaxf(max3f(m8[0], m8[1], m8[2]), max3f(max3f(m8[3], m8[4], m8[5]), m8[6], m8[7]));
         // lazy rescale: move the reference only when the max grows by > tau
@@ -346,21 +337,17 @@ INK_DEV void softmax_role(const PrefillArgs &a, float *bias_sm, uint64_t *s_full
             const f32x2 l2e2 = pk2(kLog2e, kLog2e), mneg2 = pk2(mneg, mneg);
             f32x2 acc[4] = {0ull, 0ull, 0ull, 0ull};
             uint32_t pk[64];
-            // P in two halves of 64 keys: the first half's store to tensor
-            // memory runs while the second half's exponentials are computed
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-#pragma unroll
-                for (int c = 32 * hf; c < 32 * hf + 32; ++c) {
-                    const f32x2 tt = ffma2(pk2(x[2 * c], x[2 * c + 1]), l2e2, mneg2);
-                    float t0, t1;
-                    upk2(tt, t0, t1);
-                    const float p0 = ex2(t0), p1 = ex2(t1);
-                    acc[c & 3] = fadd2(acc[c & 3], pk2(p0, p1));
-                    pk[c] = pack_bf16(p0, p1);
-                }
-                tmem_st32(s_col + 32 * hf, pk + 32 * hf);
+            for (int c = 0; c < 64; ++c) {
+                const f32x2 tt = ffma2(pk2(x[2 * c], x[2 * c + 1]), l2e2, mneg2);
+                float t0, t1;
+                upk2(tt, t0, t1);
+                const float p0 = ex2(t0), p1 = ex2(t1);
+                acc[c & 3] = fadd2(acc[c & 3], pk2(p0, p1));
+                pk[c] = pack_bf16(p0, p1);
             }
+            tmem_st32(s_col + 0, pk + 0);
+            tmem_st32(s_col + 32, pk + 32);
             const f32x2 s01 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
             float la, lb;
             upk2(s01, la, lb);
@@ -383,7 +370,7 @@ INK_DEV void softmax_role(const PrefillArgs &a, float *bias_sm, uint64_t *s_full
         tc_fence_before();
         signal_p(t);
     }
-    const bool have_o = !dead && mbar_wait_warp(&o_done[t], 0, abort_flag, a.status);
+    const bool have_o = !dead && mbar_wait_warp(&o_done[t], o_phase, abort_flag, a.status);
     if (have_o) tc_fence_after();
     epilogue(have_o, u, i, l, m_ref, o_col, abort_flag);
 }

@@ -128,8 +128,8 @@ def test_decode_swa_workload_full_size(oracle_mod):
 
 @pytest.mark.parametrize("name", ["decode_full_1m_b1", "decode_full_1m_b8"])
 def test_decode_long_context_sampled(oracle_mod, name):
-    """1M-token full-attention decode at full size; the oracle checks one query
-    head per kv head of two sequences, through a host copy of those
+    """1M-token full-attention decode at full size; the oracle checks every
+    query head of the first and last sequence, through a host copy of those
     sequences' blocks."""
     need_gpu()
     spec = WORKLOADS[name]
@@ -138,7 +138,7 @@ def test_decode_long_context_sampled(oracle_mod, name):
                           t["bias"], window=0)
     torch.cuda.synchronize()
     seqs = [0] if spec.S == 1 else [0, spec.S - 1]
-    heads = [kvh * (spec.Hq // spec.Hkv) + (kvh % 8) for kvh in range(spec.Hkv)]
+    heads = list(range(spec.Hq))
     for s in seqs:
         ids = t["block_table"][s].long()
         kc = u16(t["k_cache"][ids])                    # this sequence's blocks, in order

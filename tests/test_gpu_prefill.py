@@ -138,23 +138,27 @@ def test_prefill_last_row_equals_decode(oracle_mod):
 
 
 def _sample_rows(spec, rng, per_head):
-    """Rows that exercise every mask case: first rows, the window edge, tile
-    and query-block boundaries, the last rows, and random rows."""
+    """Stratified rows of every (batch, head): the first 128 rows, the window
+    edge W-1 .. W+128 (sliding window only), the last 128 rows, and
+    `per_head` random rows (the first query blocks, the rows where keys start
+    to leave the window, the diagonal tiles of the last query blocks, and
+    rows anywhere)."""
     T, W = spec.T, spec.window
-    fixed = [0, 1, 127, 128, 255, 256, T - 1, T - 2, T - 129]
+    fixed = list(range(0, min(128, T)))
     if W > 0:
-        fixed += [W - 1, W, W + 1, W + 127, W + 128]
-    fixed = [i for i in fixed if 0 <= i < T]
+        fixed += list(range(max(0, W - 1), min(T, W + 129)))
+    fixed += list(range(max(0, T - 128), T))
+    fixed = sorted(set(fixed))
     rows = []
     for b in range(spec.B):
         for h in range(spec.Hq):
-            pick = list(fixed) + list(rng.integers(0, T, size=per_head))
+            pick = fixed + list(rng.integers(0, T, size=per_head))
             rows += [(b, h, i) for i in pick]
     return np.array(rows, np.int32)
 
 
-@pytest.mark.parametrize("name,per_head", [("prefill_swa_b4_t8192", 4),
-                                           ("prefill_full_b1_t32768", 3)])
+@pytest.mark.parametrize("name,per_head", [("prefill_swa_b4_t8192", 256),
+                                           ("prefill_full_b1_t32768", 256)])
 def test_prefill_full_size_sampled_rows(oracle_mod, name, per_head):
     """The benchmark workloads at full size, in the benchmark's launch
     configuration; the oracle computes a sample of rows of every (batch, head)."""

@@ -104,7 +104,7 @@ def test_sharded_output_sconv_one_kernel_over_all_ranks_buffers(oracle_mod, N, T
         acc = acc + x.float()
     s = acc.to(torch.bfloat16)
     full_state = state.clone() if with_state else None
-    shards = [state[:, :, channel_shard(C, N, r)].contiguous() if with_state else None
+    shards = [state[:, :, channel_shard(C, N, r)].clone() if with_state else None
               for r in range(N)]
     for rnd in range(2):
         ys = [torch.full_like(xs[0], float("nan")) for _ in range(N)]
