@@ -78,9 +78,6 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
     const int s = blockIdx.x % a.S;
     const int kvh = (blockIdx.x / a.S) % a.Hkv;
     const int split = blockIdx.x / (a.S * a.Hkv);
-    // the combine kernel that follows (with splits) may launch now; it waits
-    // for this whole grid before reading a partial
-    if (a.splits > 1) pdl_launch_dependents();
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kDecStages; ++i) {
@@ -338,9 +335,6 @@ decode_combine_kernel(const float *__restrict__ part_o, const float *__restrict_
                       uint16_t *__restrict__ out, float *__restrict__ lse, int pairs, int splits) {
     const int pair = blockIdx.x * 4 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    // launched programmatically behind the split kernel: its partials are
-    // complete and visible only after this wait
-    pdl_wait_primary();
     if (pair >= pairs) return;
     const float *ml = part_ml + (long)pair * splits * 2;
     float M = -INFINITY;
@@ -373,24 +367,10 @@ decode_combine_kernel(const float *__restrict__ part_o, const float *__restrict_
                                : (Ls == 0.f ? -INFINITY : Ls);
 }
 
-// The combine is launched with programmatic dependent launch: its launch
-// overlaps the tail of the split kernel, which lets it start at its first
-// block, and its blocks wait for the split kernel's partials on the device.
 cudaError_t launch_decode_combine(const float *part_o, const float *part_ml, uint16_t *out, float *lse,
                                   long rows, int splits, cudaStream_t stream) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)((rows + 3) / 4), 1, 1);
-    cfg.blockDim = dim3(128, 1, 1);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, decode_combine_kernel, part_o, part_ml, out, lse,
-                                       (int)rows, splits);
-    if (e != cudaSuccess) return e;
+    decode_combine_kernel<<<(unsigned)((rows + 3) / 4), 128, 0, stream>>>(part_o, part_ml, out, lse,
+                                                                        (int)rows, splits);
     return cudaGetLastError();
 }
 

@@ -34,6 +34,24 @@ namespace inkling {
 cudaError_t launch_decode_combine(const float *part_o, const float *part_ml, uint16_t *out, float *lse,
                                   long rows, int splits, cudaStream_t stream);
 
+// A (sequence, token, head) row this call could not compute (length out of
+// range, or a bounded wait gave up) reads NaN in out and lse; with splits, a
+// NaN partial makes the merged row NaN.
+__device__ __noinline__ void decode_nan_row(uint16_t *out, float *lse, float *part_ml, int splits,
+                                            long pair, int split) {
+    const float nanv = __int_as_float(0x7fc00000);
+    if (splits == 1) {
+        const uint32_t nb = 0x7fc07fc0u;
+        uint4 *dst = (uint4 *)(out + pair * 128);
+        for (int c = 0; c < 16; ++c) dst[c] = make_uint4(nb, nb, nb, nb);
+        if (lse) lse[pair] = nanv;
+    } else {
+        const long pi = pair * splits + split;
+        part_ml[pi * 2] = nanv;
+        part_ml[pi * 2 + 1] = nanv;
+    }
+}
+
 constexpr int kMqTile = 64;                       // keys per tile (half a cache block)
 constexpr int kMqHead = 100;                      // floats per head diagonal (>= 63 + 10, == 4 mod 32)
 constexpr int kMqBiasBuf = 8 * kMqHead;
@@ -83,9 +101,6 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int kvh = (blockIdx.x / a.S) % a.Hkv;
     const int split = blockIdx.x / (a.S * a.Hkv);
     const int Q = a.Q, G = a.G, rows = G * Q;
-    // the combine kernel that follows (with splits) may launch now; it waits
-    // for this whole grid before reading a partial
-    if (a.splits > 1) pdl_launch_dependents();
 
     // key tiles of this sequence (union of its rows' windows) and this split
     const int L = a.seq_lens[s];
@@ -298,24 +313,7 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tmem_wait_ld();
         }
         auto o = [&](int i) { return __uint_as_float(ob[i]); };
-        if (rv && (bad_len || *abort_flag)) {
-            // a row this call could not compute (length out of range, or a
-            // bounded wait gave up) reads NaN; with splits, a NaN partial
-            // makes the merged row NaN
-            const long pair = ((long)s * Q + qi) * a.Hq + h;
-            const float nanv = __int_as_float(0x7fc00000);
-            if (a.splits == 1) {
-                const uint32_t nb = 0x7fc07fc0u;
-                uint4 *dst = (uint4 *)(a.out + pair * 128);
-#pragma unroll
-                for (int c = 0; c < 16; ++c) dst[c] = make_uint4(nb, nb, nb, nb);
-                if (a.lse) a.lse[pair] = nanv;
-            } else {
-                const long pi = pair * a.splits + split;
-                a.part_ml[pi * 2] = nanv;
-                a.part_ml[pi * 2 + 1] = nanv;
-            }
-        } else if (rv) {
+        if (rv && !bad_len && !*abort_flag) {
             const long pair = ((long)s * Q + qi) * a.Hq + h;
             if (a.splits == 1) {
                 const float inv = (l > 0.f) ? 1.f / l : 0.f;
@@ -437,6 +435,12 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         tc_fence_after();
         tmem_dealloc(tbase, 256);
     }
+    // rows this call could not compute read NaN: after the block's work, so
+    // that the main loop's code stays as it is without this rare path (in the
+    // epilogue it cost the kernel 6%)
+    if (warp < 4 && (int)threadIdx.x < rows && (bad_len || *abort_flag))
+        decode_nan_row(a.out, a.lse, a.part_ml, a.splits,
+                       ((long)s * Q + threadIdx.x / G) * a.Hq + kvh * G + threadIdx.x % G, split);
 }
 
 cudaError_t launch_attn_decode_mq(const inkling_decode_params &p, int splits, void *workspace,

@@ -163,7 +163,10 @@ attn_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
 
     if (warp < 8) {
         // ================================================== softmax (2 WGs) ==
-        setmaxnreg_inc184();
+        if (kFill)
+            setmaxnreg_inc168();
+        else
+            setmaxnreg_inc184();
         const int t = warp >> 2;
         if (ok[t])
             softmax_role(a, (float *)(smem + PBIAS) + t * 2 * kBiasBuf, &bar[S_FULL], &bar[O_DONE],
@@ -175,7 +178,10 @@ attn_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                          TmaStoreEpilogue{a, smem + PQ + t * 32768, &tm_out, b, hd[t], r0[t], 3 + t});
     } else if (warp < 12) {
         // ==================== sconv of this CTA's halves: warps 8-9 keys, 10-11 values ==
-        setmaxnreg_dec80();
+        if (kFill)
+            setmaxnreg_dec96();
+        else
+            setmaxnreg_dec80();
         const bool is_v = warp >= 10;
         const int v = threadIdx.x - (is_v ? 320 : 256);
         const int bar_id = is_v ? 2 : 1;
@@ -215,7 +221,10 @@ attn_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
             mbar_arrive_cta(&ready[st], 0);
         }
     } else {
-        setmaxnreg_dec64();
+        if (kFill)
+            setmaxnreg_dec80();
+        else
+            setmaxnreg_dec64();
         if (kFill && warp == 14 && rank == 0 && hsel == 0 && f.k_state &&
             uhi == (a.T - 1) >> 7) {
             // the new sconv state, by the block that owns the last key tile

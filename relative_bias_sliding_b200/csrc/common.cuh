@@ -359,15 +359,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major, 
            ((uint32_t)(M >> 4) << 24);
 }
 
-// ------------------------------------------- programmatic dependent launch --
-// A kernel launched with the programmatic-stream-serialization attribute may
-// start while the kernel before it on the stream is still running; it waits
-// here until that kernel has completed and its memory operations are visible.
-INK_DEV void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-// Let the dependent kernel of the stream launch now (its blocks then wait in
-// pdl_wait_primary for this whole grid); issued by each block at its start.
-INK_DEV void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-
 // ------------------------------------------------------------- numerics --
 
 INK_DEV float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }

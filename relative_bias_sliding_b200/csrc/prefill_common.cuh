@@ -74,6 +74,14 @@ INK_DEV void write_sconv_state(const FillArgs &f, const PrefillArgs &a, int b, i
 INK_DEV void setmaxnreg_inc184() { asm volatile("setmaxnreg.inc.sync.aligned.u32 184;"); }
 INK_DEV void setmaxnreg_dec80() { asm volatile("setmaxnreg.dec.sync.aligned.u32 80;"); }
 INK_DEV void setmaxnreg_dec64() { asm volatile("setmaxnreg.dec.sync.aligned.u32 64;"); }
+// The split of the cache-filling CTA-pair prefill: its sconv warps also store
+// the converted tiles to the paged cache, and its producer / MMA group tracks
+// the fill, so they get 96 and 80 registers and the softmax groups 168:
+// 2 x 128 x 168 + 128 x 96 + 128 x 80 = 65536.  Measured on the
+// sliding-window workload: 687 TFLOP/s against 655 with the plain split (the
+// plain prefill keeps its split: 696 against 689).
+INK_DEV void setmaxnreg_inc168() { asm volatile("setmaxnreg.inc.sync.aligned.u32 168;"); }
+INK_DEV void setmaxnreg_dec96() { asm volatile("setmaxnreg.dec.sync.aligned.u32 96;"); }
 
 // Taps of 8 consecutive channels starting at `wg` ([C, 4] fp32), as channel
 // pairs: w[tap][p] = (w[2p][tap], w[2p+1][tap]).
