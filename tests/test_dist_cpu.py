@@ -135,3 +135,30 @@ def test_channel_sharded_output_sconv_gloo_world2():
         assert (y == _bits(y_ref)).all(), f"rank {r}: first call"
         assert (y2 == _bits(y2_ref)).all(), f"rank {r}: second call"
         assert (st == _bits(state[:, :, channel_shard(C, world, r)])).all(), f"rank {r}: state"
+
+
+def test_shard_selection_covers_every_head_and_channel_once():
+    """kv_head_shard / channel_shard: the ranks' slices tile the heads and the
+    channels exactly once, in order, and each rank's query heads are the ones
+    that read its kv heads (contiguous grouping h -> h / (Hq / Hkv))."""
+    sys.path.insert(0, ROOT)
+    from relative_bias_sliding_b200.sharded import channel_shard, kv_head_shard
+    for Hq, Hkv, world in [(64, 8, 1), (64, 8, 2), (64, 8, 4), (64, 8, 8), (16, 4, 2), (6, 2, 2)]:
+        G = Hq // Hkv
+        qs, ks, cs = [], [], []
+        for r in range(world):
+            q, k, c = kv_head_shard(Hq, Hkv, world, r)
+            qs += list(range(Hq))[q]
+            ks += list(range(Hkv))[k]
+            cs += list(range(Hkv * 128))[c]
+            assert all(h // G in list(range(Hkv))[k] for h in list(range(Hq))[q])
+        assert qs == list(range(Hq)) and ks == list(range(Hkv)) and cs == list(range(Hkv * 128))
+    for C, world in [(1024, 1), (1024, 2), (8192, 8)]:
+        got = []
+        for r in range(world):
+            got += list(range(C))[channel_shard(C, world, r)]
+        assert got == list(range(C))
+    with pytest.raises(ValueError):
+        kv_head_shard(64, 8, 3, 0)       # 8 kv heads over 3 ranks
+    with pytest.raises(ValueError):
+        channel_shard(1000, 2, 0)        # channels not a multiple of 8 * ranks
