@@ -483,6 +483,10 @@ static inkling_status decode_with(const inkling_decode_params *p, int splits, vo
         return fail(INKLING_ERR_UNSUPPORTED, "num_seqs * num_kv_heads * splits (%d) exceeds 2^31",
                     splits);
     if (splits > 1) {
+        // the combine pass runs one thread block per output row
+        if ((long)decode_rows(*p) * p->num_q_heads >= (1L << 31))
+            return fail(INKLING_ERR_UNSUPPORTED, "%ld output rows to combine exceed 2^31",
+                        (long)decode_rows(*p) * p->num_q_heads);
         const size_t need = inkling_attn_decode_workspace_bytes(decode_rows(*p), p->num_q_heads, splits);
         if (!workspace || workspace_bytes < need)
             return fail(INKLING_ERR_INVALID, "workspace of %zu bytes given, %zu needed for %d splits",
