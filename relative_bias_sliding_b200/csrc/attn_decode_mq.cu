@@ -9,9 +9,10 @@
 // head) rows of the kv head (at most 80) form one 128-row tile: a single 3-D
 // TMA box gathers them (q viewed as [S*q_len, Hq, d], box {64, G, q_len}),
 // rows ordered r = qi*G + g.  Key tiles are 64 tokens, half a cache block
-// (two 64-column TMA boxes each for keys and values, 128-byte swizzle), so a
-// block needs ~105 KB of shared memory and 256 TMEM columns and two blocks
-// share an SM: one's softmax runs while the other waits on its tiles.
+// (two 64-column TMA boxes each for keys and values, 128-byte swizzle), keys
+// in 3 stages and values in 2, so a block needs ~108 KB of shared memory and
+// 256 TMEM columns and two blocks share an SM: one's softmax runs while the
+// other waits on its tiles.
 //   S = Q K^T: tcgen05 M=128 N=64 into one of two TMEM buffers, so the MMA
 //     of key tile k+1 runs while the softmax works on tile k;
 //   P (bf16) over the first 32 columns of its S buffer; O += P V (TMEM A);
@@ -55,25 +56,30 @@ __device__ __noinline__ void decode_nan_row(uint16_t *out, float *lse, float *pa
 constexpr int kMqTile = 64;                       // keys per tile (half a cache block)
 constexpr int kMqHead = 100;                      // floats per head diagonal (>= 63 + 10, == 4 mod 32)
 constexpr int kMqBiasBuf = 8 * kMqHead;
-constexpr uint32_t MQ_Q = 0;                      // 128 rows x 256 B (two 16 KB halves)
-constexpr uint32_t MQ_K = 32768;                  // 2 stages x 16 KB (two 64-row d halves)
-constexpr uint32_t MQ_V = 65536;                  // 2 stages x 16 KB
-constexpr uint32_t MQ_BIAS = 98304;               // 2 buffers of staged diagonals
+// The query tile holds at most 80 rows (two 10 KB d halves).  The M=128 MMA
+// also reads rows 80..127 of each half, which lie in the next half or in the
+// first key stage: those rows' S, P and O are never used.
+constexpr uint32_t kMqQHalf = 10240;              // 80 rows x 128 B
+constexpr int kMqKStages = 3;                     // keys: 3 stages, values: 2
+constexpr uint32_t MQ_Q = 0;
+constexpr uint32_t MQ_K = 2 * kMqQHalf;           // 3 stages x 16 KB (two 64-row d halves)
+constexpr uint32_t MQ_V = MQ_K + kMqKStages * 16384;  // 2 stages x 16 KB
+constexpr uint32_t MQ_BIAS = MQ_V + 2 * 16384;    // 2 buffers of staged diagonals
 constexpr uint32_t MQ_BAR = MQ_BIAS + 2 * kMqBiasBuf * 4;
 constexpr int kMqSmem = MQ_BAR + 256 + 1024;
 
 enum {
     M_QFULL = 0,
-    M_KFULL = 1,    // +stage
-    M_VFULL = 3,
-    M_KEMPTY = 5,
-    M_VEMPTY = 7,
-    M_SFULL = 9,    // +S buffer
-    M_PFULL = 11,   // +S buffer (128 arrivals)
-    M_OREADY = 13,  // one phase per P.V issued
-    M_DRAIN = 14,
-    M_ODONE = 15,   // the last P.V has completed (one phase)
-    M_COUNT = 16
+    M_KFULL = 1,    // +key stage
+    M_VFULL = 4,    // +value stage
+    M_KEMPTY = 6,
+    M_VEMPTY = 9,
+    M_SFULL = 11,   // +S buffer
+    M_PFULL = 13,   // +S buffer (128 arrivals)
+    M_OREADY = 15,  // one phase per P.V issued
+    M_DRAIN = 16,
+    M_ODONE = 17,   // the last P.V has completed (one phase)
+    M_COUNT = 18
 };
 
 struct DecodeMqArgs {
@@ -206,11 +212,14 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tmem_ld32(s_col + 0, sr + 0);
             tmem_ld32(s_col + 32, sr + 32);
             tmem_wait_ld();
-            // columns this row may see: ipos - j0 - c in [0, W)
+            // columns this row may see: ipos - j0 - c in [0, W).  The choice
+            // of path is warp-uniform and padding rows (whose S, P and O are
+            // never read) take no part in it: a warp that held both paths ran
+            // both, one after the other
             const int dist0 = ipos - j0;
-            const int cmax = rv ? min(kMqTile - 1, dist0) : -1;
-            const int cmin = (W > 0) ? max(0, dist0 - W + 1) : 0;
-            const bool full = cmin == 0 && cmax == kMqTile - 1;
+            const int cmax = rv ? min(kMqTile - 1, dist0) : kMqTile - 1;
+            const int cmin = (rv && W > 0) ? max(0, dist0 - W + 1) : 0;
+            const bool full = __all_sync(0xffffffffu, cmin == 0 && cmax == kMqTile - 1);
             const float *rb = bb + g * kMqHead + o_rd;
             float x[64];
             float m8[8];
@@ -249,7 +258,7 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 logits(std::true_type{});
             const float mx =
                 fmaxf(max3f(m8[0], m8[1], m8[2]), max3f(max3f(m8[3], m8[4], m8[5]), m8[6], m8[7]));
-            const bool grow = mx > m_ref + kTau;
+            const bool grow = rv && mx > m_ref + kTau;
             float alpha = 1.f;
             if (grow) {
                 alpha = ex2((m_ref - mx) * kLog2e);
@@ -349,45 +358,58 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (nt > 0) {
             mbar_arrive_expect_tx(&bar[M_QFULL], 2 * rows * 128);
             tma_load_3d(smem + MQ_Q, &tm_q, &bar[M_QFULL], 0, kvh * G, s * Q);
-            tma_load_3d(smem + MQ_Q + 16384, &tm_q, &bar[M_QFULL], 64, kvh * G, s * Q);
+            tma_load_3d(smem + MQ_Q + kMqQHalf, &tm_q, &bar[M_QFULL], 64, kvh * G, s * Q);
         }
-        int issued = 0;
-        for (int k = 0; k < nt; ++k) {
-            const int st = k & 1;
-            const uint32_t ph = ((k >> 1) & 1) ^ 1;
+        // cache row of key tile k (half n % 2 of cache block n / 2)
+        auto tile_row = [&](int k) {
             int blk = a.block_table[(long)s * a.max_blocks + (ta + k) / 2];
             if (blk < 0 || blk >= a.num_blocks) {
                 report_status(a.status, INKLING_STATUS_BAD_BLOCK);
                 blk = 0;  // keep the pipeline running on a valid block
             }
-            const int n = ta + k;  // key tile: half n % 2 of cache block n / 2
-            const int row = (blk * a.Hkv + kvh) * 128 + (n & 1) * kMqTile;
-            if (!mbar_wait(&bar[M_KEMPTY + st], ph, abort_flag, a.status)) break;
-            mbar_arrive_expect_tx(&bar[M_KFULL + st], 16384);
-            tma_load_2d(smem + MQ_K + st * 16384, &tm_k, &bar[M_KFULL + st], 0, row);
-            tma_load_2d(smem + MQ_K + st * 16384 + 8192, &tm_k, &bar[M_KFULL + st], 64, row);
-            if (!mbar_wait(&bar[M_VEMPTY + st], ph, abort_flag, a.status)) break;
-            mbar_arrive_expect_tx(&bar[M_VFULL + st], 16384);
-            tma_load_2d(smem + MQ_V + st * 16384, &tm_v, &bar[M_VFULL + st], 0, row);
-            tma_load_2d(smem + MQ_V + st * 16384 + 8192, &tm_v, &bar[M_VFULL + st], 64, row);
-            ++issued;
+            return (blk * a.Hkv + kvh) * 128 + ((ta + k) & 1) * kMqTile;
+        };
+        // Loads in the order their stages free up: K0 K1 K2 V0 K3 V1 K4 V2 ...
+        // V(k) waits for P.V(k-2), K(k+3) for QK^T(k), and the MMA runs
+        // QK^T(k) before P.V(k-1).  Keys are fetched three tiles ahead, values
+        // two.
+        int kk = 0, vv = 0;
+        while (kk < nt || vv < nt) {
+            if (kk < nt && kk < vv + kMqKStages) {
+                const int st = kk % kMqKStages;
+                const int row = tile_row(kk);
+                if (!mbar_wait(&bar[M_KEMPTY + st], ((kk / kMqKStages) & 1) ^ 1, abort_flag, a.status))
+                    break;
+                mbar_arrive_expect_tx(&bar[M_KFULL + st], 16384);
+                tma_load_2d(smem + MQ_K + st * 16384, &tm_k, &bar[M_KFULL + st], 0, row);
+                tma_load_2d(smem + MQ_K + st * 16384 + 8192, &tm_k, &bar[M_KFULL + st], 64, row);
+                ++kk;
+            } else {
+                const int st = vv & 1;
+                const int row = tile_row(vv);
+                if (!mbar_wait(&bar[M_VEMPTY + st], ((vv >> 1) & 1) ^ 1, abort_flag, a.status)) break;
+                mbar_arrive_expect_tx(&bar[M_VFULL + st], 16384);
+                tma_load_2d(smem + MQ_V + st * 16384, &tm_v, &bar[M_VFULL + st], 0, row);
+                tma_load_2d(smem + MQ_V + st * 16384 + 8192, &tm_v, &bar[M_VFULL + st], 64, row);
+                ++vv;
+            }
         }
         // drain: every load issued has landed before the block may exit
         if (nt > 0) mbar_wait(&bar[M_QFULL], 0, nullptr, a.status);
-        for (int k = max(0, issued - 2); k < issued; ++k) {
-            mbar_wait(&bar[M_KFULL + (k & 1)], (k >> 1) & 1, nullptr, a.status);
+        for (int k = max(0, kk - kMqKStages); k < kk; ++k)
+            mbar_wait(&bar[M_KFULL + k % kMqKStages], (k / kMqKStages) & 1, nullptr, a.status);
+        for (int k = max(0, vv - 2); k < vv; ++k)
             mbar_wait(&bar[M_VFULL + (k & 1)], (k >> 1) & 1, nullptr, a.status);
-        }
     } else if (warp == 5 && lane == 0) {
         // ================================================ MMA issuer ==
         const uint32_t id_qk = idesc_bf16(128, kMqTile, 0, 0);
         const uint32_t id_pv = idesc_bf16(128, 128, 0, 1);
         auto issue_qk = [&](int k) {
-            const int st = k & 1;
+            const int st = k % kMqKStages;
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint64_t ad =
-                    sw128_desc(sb + MQ_Q + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+                    sw128_desc(sb + MQ_Q + (ks >> 2) * kMqQHalf + (ks & 3) * 32, 16, 1024);
                 const uint64_t bd =
                     sw128_desc(sb + MQ_K + st * 16384 + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
                 umma_ss(tbase + (k & 1) * kMqTile, ad, bd, id_qk, ks > 0 ? 1u : 0u);
@@ -407,11 +429,13 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // tile runs while the softmax works on the current one
         for (int k = 0; k <= nt && alive; ++k) {
             if (k < nt) {
-                if (!mbar_wait(&bar[M_KFULL + (k & 1)], (k >> 1) & 1, abort_flag, a.status)) break;
+                if (!mbar_wait(&bar[M_KFULL + k % kMqKStages], (k / kMqKStages) & 1, abort_flag,
+                               a.status))
+                    break;
                 tc_fence_after();
                 issue_qk(k);
                 tc_commit(&bar[M_SFULL + (k & 1)]);
-                tc_commit(&bar[M_KEMPTY + (k & 1)]);
+                tc_commit(&bar[M_KEMPTY + k % kMqKStages]);
             }
             if (k >= 1) {
                 const int kp = k - 1;
