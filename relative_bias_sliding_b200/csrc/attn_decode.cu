@@ -329,65 +329,78 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
     __syncthreads();
 }
 
-// One block per (sequence, query head) row: log-sum-exp merge of the splits.
-// Each of the 8 warps takes every 8th split (lane l holds dims 4l..4l+3),
-// four splits' loads in flight at a time, and the warps' sums meet in shared
-// memory in a fixed order.  A warp per row walking all splits in turn was
-// latency-bound: 45 us for 64 rows x 148 splits (1M-token decode, batch 1),
-// 6% of that step; the whole step went from 0.710 to 0.682 ms.
+// Log-sum-exp merge of the splits of each (sequence, token, query head) row.
+// A block of 8 warps merges 8 / WPR rows, WPR warps per row: warp w of a row
+// takes every WPR-th split (lane l holds dims 4l..4l+3) with four splits'
+// loads in flight, and the row's warps meet in shared memory in a fixed
+// order.  WPR grows with the split count (1 below 8 splits, 8 from 32 on).  A
+// single warp per row walking 148 splits in turn was latency-bound: 45 us for
+// the 64 rows of a 1M-token batch-1 decode, 6% of that step (0.710 -> 0.682
+// ms with 8 warps per row).
 constexpr int kCombWarps = 8;
 
+template <int WPR>
 __global__ void __launch_bounds__(kCombWarps * 32)
 decode_combine_kernel(const float *__restrict__ part_o, const float *__restrict__ part_ml,
-                      uint16_t *__restrict__ out, float *__restrict__ lse, int splits) {
+                      uint16_t *__restrict__ out, float *__restrict__ lse, long rows, int splits) {
     __shared__ float s_m[kCombWarps];
     __shared__ float s_ls[kCombWarps];
     __shared__ float4 s_acc[kCombWarps][32];
-    const long pair = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const float *ml = part_ml + pair * splits * 2;
+    const int sub = warp % WPR, w0 = warp - sub;  // this row's first warp
+    const long pair = (long)blockIdx.x * (kCombWarps / WPR) + warp / WPR;
+    const bool live = pair < rows;
+    const float *ml = part_ml + (live ? pair : 0) * splits * 2;
     float M = -INFINITY;
-    for (int sp = threadIdx.x; sp < splits; sp += kCombWarps * 32) M = fmaxf(M, ml[sp * 2]);
+    if (live)
+        for (int sp = sub * 32 + lane; sp < splits; sp += WPR * 32) M = fmaxf(M, ml[sp * 2]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    if (lane == 0) s_m[warp] = M;
-    __syncthreads();
+    if (WPR > 1) {
+        if (lane == 0) s_m[warp] = M;
+        __syncthreads();
 #pragma unroll
-    for (int w = 0; w < kCombWarps; ++w) M = fmaxf(M, s_m[w]);
+        for (int w = 0; w < WPR; ++w) M = fmaxf(M, s_m[w0 + w]);
+    }
     float Ls = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    const float4 *po = (const float4 *)(part_o + pair * splits * 128) + lane;
+    const float4 *po = (const float4 *)(part_o + (live ? pair : 0) * splits * 128) + lane;
+    if (live) {
 #pragma unroll 4
-    for (int sp = warp; sp < splits; sp += kCombWarps) {
-        const float msp = ml[sp * 2];
-        const float lsp = ml[sp * 2 + 1];
-        const float4 v = po[sp * 32];
-        // an empty split (no key in range) carries m = -inf and takes no
-        // weight; a NaN partial passes into Ls and the output
-        if (msp != -INFINITY) {
-            const float f = ex2(msp - M);
-            Ls = fmaf(f, lsp, Ls);
-            acc.x = fmaf(f, v.x, acc.x);
-            acc.y = fmaf(f, v.y, acc.y);
-            acc.z = fmaf(f, v.z, acc.z);
-            acc.w = fmaf(f, v.w, acc.w);
+        for (int sp = sub; sp < splits; sp += WPR) {
+            const float msp = ml[sp * 2];
+            const float lsp = ml[sp * 2 + 1];
+            const float4 v = po[sp * 32];
+            // an empty split (no key in range) carries m = -inf and takes no
+            // weight; a NaN partial passes into Ls and the output
+            if (msp != -INFINITY) {
+                const float f = ex2(msp - M);
+                Ls = fmaf(f, lsp, Ls);
+                acc.x = fmaf(f, v.x, acc.x);
+                acc.y = fmaf(f, v.y, acc.y);
+                acc.z = fmaf(f, v.z, acc.z);
+                acc.w = fmaf(f, v.w, acc.w);
+            }
         }
     }
-    s_acc[warp][lane] = acc;
-    if (lane == 0) s_ls[warp] = Ls;
-    __syncthreads();
-    if (warp != 0) return;
-    acc = s_acc[0][lane];
-    Ls = s_ls[0];
+    if (WPR > 1) {
+        s_acc[warp][lane] = acc;
+        if (lane == 0) s_ls[warp] = Ls;
+        __syncthreads();
+        if (sub != 0) return;
+        acc = s_acc[w0][lane];
+        Ls = s_ls[w0];
 #pragma unroll
-    for (int w = 1; w < kCombWarps; ++w) {
-        const float4 b = s_acc[w][lane];
-        acc.x += b.x;
-        acc.y += b.y;
-        acc.z += b.z;
-        acc.w += b.w;
-        Ls += s_ls[w];
+        for (int w = 1; w < WPR; ++w) {
+            const float4 b = s_acc[w0 + w][lane];
+            acc.x += b.x;
+            acc.y += b.y;
+            acc.z += b.z;
+            acc.w += b.w;
+            Ls += s_ls[w0 + w];
+        }
     }
+    if (!live) return;
     // a NaN partial makes Ls, the output and the lse NaN
     const float inv = (Ls > 0.f) ? 1.f / Ls : 0.f;
     uint2 pk;
@@ -399,12 +412,22 @@ decode_combine_kernel(const float *__restrict__ part_o, const float *__restrict_
                                : (Ls == 0.f ? -INFINITY : Ls);
 }
 
+template <int WPR>
+static cudaError_t launch_combine_wpr(const float *part_o, const float *part_ml, uint16_t *out,
+                                      float *lse, long rows, int splits, cudaStream_t stream) {
+    const long per = kCombWarps / WPR;
+    decode_combine_kernel<WPR><<<(unsigned)((rows + per - 1) / per), kCombWarps * 32, 0, stream>>>(
+        part_o, part_ml, out, lse, rows, splits);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_decode_combine(const float *part_o, const float *part_ml, uint16_t *out, float *lse,
                                   long rows, int splits, cudaStream_t stream) {
     if (rows == 0) return cudaSuccess;
-    decode_combine_kernel<<<(unsigned)rows, kCombWarps * 32, 0, stream>>>(part_o, part_ml, out, lse,
-                                                                          splits);
-    return cudaGetLastError();
+    if (splits >= 32) return launch_combine_wpr<8>(part_o, part_ml, out, lse, rows, splits, stream);
+    if (splits >= 16) return launch_combine_wpr<4>(part_o, part_ml, out, lse, rows, splits, stream);
+    if (splits >= 8) return launch_combine_wpr<2>(part_o, part_ml, out, lse, rows, splits, stream);
+    return launch_combine_wpr<1>(part_o, part_ml, out, lse, rows, splits, stream);
 }
 
 cudaError_t launch_attn_decode(const inkling_decode_params &p, int splits, void *workspace,
