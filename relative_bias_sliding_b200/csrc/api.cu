@@ -113,13 +113,18 @@ static int32_t decode_rows(const inkling_decode_params &p) {
 
 // Split count for num_splits = 0.  Both decode kernels run two blocks per SM
 // (`slots` = 2 x SMs).  When the (sequence, kv head) units alone fill the
-// slots the key range is not split (no partials, no combine pass).
-// Otherwise the count starts at about 8 blocks per SM and, within twice that,
-// takes the one whose last wave is fullest, with at least ~512 keys (8
-// chunks) per split.  Measured on B200: 64 sequences x 8 kv heads, window
-// 4096: 1 split 6.13 TB/s vs 3 splits 5.63; 1M tokens x 8 sequences: 37
-// splits (8 full waves) 6.7 TB/s vs 19 splits 5.9; 1M x 1: 148 splits 6.06 vs
-// 296 splits 5.56.
+// slots the key range is not split (no partials, no combine pass).  A short
+// key range (at most 4096 keys per split) takes one wave: as many splits as
+// fit in the slots, at least ~512 keys (8 chunks) each.  A long one starts at
+// about 8 blocks per SM and, within twice that, takes the count whose last
+// wave is fullest.  Measured on B200 (KV GB/s):
+//   window 4096, 1 token:  8 seqs  4 splits 3839, 8 splits ~3000;
+//                         16 seqs  2 splits 4774, 4: 4554, 8: 4150;
+//                         32 seqs  1 split  5745, 2: 5458;
+//   window 4096, 9 tokens: 8 seqs  4 splits 2882, 8: 2539;
+//                         16 seqs  2 splits 3735, 8: 2940;  32 seqs 1 split 4574;
+//   1M tokens, 1 token:  batch 8 37 splits (8 full waves) 6716 vs 19: 6081;
+//                        batch 1 148 splits 6309 vs 222: 6262.
 int decode_splits(const inkling_decode_params &p, int num_sms) {
     if (p.num_splits > 0) return p.num_splits;
     const long units = (long)p.num_seqs * p.num_kv_heads;
@@ -131,6 +136,8 @@ int decode_splits(const inkling_decode_params &p, int num_sms) {
     long cap = chunks / 8;
     if (cap < 1) cap = 1;
     if (cap > 1024) cap = 1024;
+    const long one_wave = slots / units;
+    if (keys <= 4096L * one_wave) return (int)(one_wave < cap ? one_wave : cap);
     long s0 = (4 * slots + units - 1) / units;
     if (s0 > cap) s0 = cap;
     long best = s0;

@@ -92,14 +92,14 @@ def test_static_scratch_decode_matches_oracle(oracle_mod, window):
 
 
 def test_static_scratch_lowers_the_automatic_split_count(oracle_mod):
-    """Multi-token decode (4 draft tokens) of 2 sequences of 40,000 tokens:
+    """Multi-token decode (10 draft tokens) of 2 sequences of 40,000 tokens:
     the automatic split count needs more partials than the 8 MiB array holds,
     so the call lowers it to the largest count that fits.  Checked against
     inkling_attn_decode with a workspace at that count (same kernels, same
     result bit for bit) and against the oracle on every row."""
     need_gpu()
     spec = scaled(WORKLOADS["decode_swa_s64"], S=2, L_min=40000, L_max=40000, window=0,
-                  D_max=65536, n_new=4, seed=22)
+                  D_max=65536, n_new=10, seed=22)
     t = make_decode(spec, device="cuda")
     S, Q, Hq = spec.S, spec.n_new, spec.Hq
     auto = ink.decode_num_splits(t["q"], t["k_cache"], t["v_cache"], t["block_table"],
