@@ -53,6 +53,7 @@ MEASURED_TRAFFIC = {
     "prefill_swa_b4_t8192": 678_828_544 + 502_533_120,
     "prefill_paged_swa_b4_t8192": 676_309_248 + 497_455_616,
     "decode_swa_s64": 1_080_856_064 + 4_138_752,
+    "decode_mtp9_swa_s64": 1_089_919_744 + 8_944_640,
 }
 
 

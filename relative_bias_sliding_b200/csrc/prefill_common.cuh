@@ -291,7 +291,9 @@ INK_DEV void softmax_role(const PrefillArgs &a, float *bias_sm, uint64_t *s_full
         // dist0 - c >= 0, dist0 - c < W (when windowed) and j0 + c < T
         const int cmax = min(min(127, dist0), T - 1 - j0);
         const int cmin = (W > 0) ? max(0, dist0 - W + 1) : 0;
-        const bool full = cmin == 0 && cmax == 127;
+        // one path per warp: a warp holding both would run both (rows of a
+        // window or chunk edge that falls inside the warp)
+        const bool full = __all_sync(0xffffffffu, cmin == 0 && cmax == 127);
         // logits and row max, 32 columns at a time: the 8 bias loads of a batch
         // are issued together, and 8 independent 3-input max chains run
         // alongside.  Rows of a partial tile take the same paired FMAs and then
