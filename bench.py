@@ -312,72 +312,112 @@ def timed_loop(steps, fns, stream):
             for i in range(len(fns))]
 
 
+def pipelined_steps(steps, h2d, compute, d2h, stream):
+    """Time ``steps`` end-to-end steps as a server runs them: step i's inputs
+    copy in (pinned host -> device, own stream) while step i-1 computes and
+    step i-2's result copies out (device -> pinned host, own stream).  Device
+    buffers are double-buffered by step parity; events order each buffer's
+    reuse.  Every step's copies fall inside the timed region, which starts
+    before the first copy-in and ends after the last copy-out.  Returns mean
+    milliseconds per step."""
+    import torch
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+    in_done, comp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+
+    def issue(i):
+        b = i & 1
+        if i >= 2:
+            s_in.wait_event(comp_done[b])  # step i-2 has finished reading inputs[b]
+        h2d(b, s_in)
+        in_done[b].record(s_in)
+        stream.wait_event(in_done[b])
+        if i >= 2:
+            stream.wait_event(out_done[b])  # step i-2's result has left outputs[b]
+        compute(b, stream)
+        comp_done[b].record(stream)
+        s_out.wait_event(comp_done[b])
+        d2h(b, s_out)
+        out_done[b].record(s_out)
+
+    for i in range(2):  # warm-up through both buffers
+        issue(i)
+    torch.cuda.synchronize()
+    a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    s_in.wait_event(a)
+    for i in range(steps):
+        issue(i)
+    stream.wait_event(out_done[(steps - 1) & 1])
+    z.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(z) / steps
+
+
 def e2e_prefill(step, steps, stream):
     """Same prefill through the public API with host buffers: pinned host ->
-    device copies of the step's inputs, the call, and the output read back."""
+    device copies of the step's inputs, the call, and the output read back,
+    pipelined across steps (pipelined_steps)."""
     import torch
     t = step.t
     host = {k: t[k].cpu().pin_memory() for k in ("q", "k_raw", "v_raw")}
     out_h = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
-    dev = {k: torch.empty_like(t[k]) for k in host}
+    dev = [{k: torch.empty_like(t[k]) for k in host} for _ in range(2)]
+    outs = [step.out, torch.empty_like(step.out)]
     import relative_bias_sliding_b200 as ink
 
-    def once():
-        for k in host:
-            dev[k].copy_(host[k], non_blocking=True)
-        ink.attn_prefill(dev["q"], dev["k_raw"], dev["v_raw"], t["w_k"], t["w_v"], t["bias"],
-                         window=step.spec.window, out=step.out, stream=stream)
-        out_h.copy_(step.out, non_blocking=True)
+    def h2d(b, s):
+        with torch.cuda.stream(s):
+            for k in host:
+                dev[b][k].copy_(host[k], non_blocking=True)
 
-    with torch.cuda.stream(stream):
-        once()
-        stream.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(steps):
-            once()
-        b.record(stream)
-        stream.synchronize()
-    ms = a.elapsed_time(b) / steps
-    h2d = sum(v.numel() * v.element_size() for v in host.values())
-    return ms, h2d, out_h.numel() * out_h.element_size()
+    def compute(b, s):
+        ink.attn_prefill(dev[b]["q"], dev[b]["k_raw"], dev[b]["v_raw"], t["w_k"], t["w_v"],
+                         t["bias"], window=step.spec.window, out=outs[b], stream=s)
+
+    def d2h(b, s):
+        with torch.cuda.stream(s):
+            out_h.copy_(outs[b], non_blocking=True)
+
+    ms = pipelined_steps(steps, h2d, compute, d2h, stream)
+    h2d_bytes = sum(v.numel() * v.element_size() for v in host.values())
+    return ms, h2d_bytes, out_h.numel() * out_h.element_size()
 
 
 def e2e_decode(step, steps, stream):
     """Decode step through the public API with host buffers for the per-step
-    inputs (queries, new raw keys/values, lengths, block table); the caches
-    and sconv states stay resident as the layer's state."""
+    inputs (queries, new raw keys/values, lengths, block table), pipelined
+    across steps (pipelined_steps); the caches and sconv states stay resident
+    as the layer's state."""
     import torch
     t = step.t
     names = ("q", "k_new", "v_new", "seq_lens", "block_table")
     host = {k: t[k].cpu().pin_memory() for k in names}
     out_h = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
-    dev = {k: torch.empty_like(t[k]) for k in names}
+    dev = [{k: torch.empty_like(t[k]) for k in names} for _ in range(2)]
+    outs = [step.out, torch.empty_like(step.out)]
     import relative_bias_sliding_b200 as ink
 
-    def once():
-        for k in names:
-            dev[k].copy_(host[k], non_blocking=True)
-        ink.sconv_kv(dev["k_new"], dev["v_new"], t["w_k"], t["w_v"], t["k_state"], t["v_state"],
-                     t["k_cache"], t["v_cache"], dev["block_table"], dev["seq_lens"],
-                     stream=stream)
-        ink.attn_decode(dev["q"], t["k_cache"], t["v_cache"], dev["block_table"],
-                        dev["seq_lens"], t["bias"], window=step.spec.window, out=step.out,
-                        workspace=step.ws, num_splits=step.splits, stream=stream)
-        out_h.copy_(step.out, non_blocking=True)
+    def h2d(b, s):
+        with torch.cuda.stream(s):
+            for k in names:
+                dev[b][k].copy_(host[k], non_blocking=True)
 
-    with torch.cuda.stream(stream):
-        once()
-        stream.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(steps):
-            once()
-        b.record(stream)
-        stream.synchronize()
-    ms = a.elapsed_time(b) / steps
-    h2d = sum(v.numel() * v.element_size() for v in host.values())
-    return ms, h2d, out_h.numel() * out_h.element_size()
+    def compute(b, s):
+        d = dev[b]
+        ink.sconv_kv(d["k_new"], d["v_new"], t["w_k"], t["w_v"], t["k_state"], t["v_state"],
+                     t["k_cache"], t["v_cache"], d["block_table"], d["seq_lens"], stream=s)
+        ink.attn_decode(d["q"], t["k_cache"], t["v_cache"], d["block_table"], d["seq_lens"],
+                        t["bias"], window=step.spec.window, out=outs[b], workspace=step.ws,
+                        num_splits=step.splits, stream=s)
+
+    def d2h(b, s):
+        with torch.cuda.stream(s):
+            out_h.copy_(outs[b], non_blocking=True)
+
+    ms = pipelined_steps(steps, h2d, compute, d2h, stream)
+    h2d_bytes = sum(v.numel() * v.element_size() for v in host.values())
+    return ms, h2d_bytes, out_h.numel() * out_h.element_size()
 
 
 # ------------------------------------------------------------ CPU oracle --
