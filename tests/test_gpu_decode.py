@@ -88,6 +88,20 @@ def test_decode_block_permutation_is_bit_exact():
     assert torch.equal(out1, out2)
 
 
+@pytest.mark.parametrize("splits", [8, 12, 20, 40])
+def test_decode_combine_warps_per_row_matches_oracle(oracle_mod, splits):
+    """The combine merges each row with 1, 2, 4 or 8 warps by split count:
+    each width against the oracle, with empty splits (a 130-token sequence)
+    in the mix."""
+    need_gpu()
+    lens = [9000, 130, 20000]
+    t, W = _inputs(3, lens, Hq=16, Hkv=2, window=0, d_max=30000, seed=40 + splits)
+    ref, ref_lse = _oracle(oracle_mod, t, W)
+    out, lse = _gpu(t, W, splits)
+    assert_parity(out, ref, f"splits={splits}")
+    np.testing.assert_allclose(lse.cpu().numpy().reshape(-1), ref_lse, rtol=0, atol=2e-3)
+
+
 def test_decode_split_count_invariance():
     need_gpu()
     lens = [9000, 130, 4500]

@@ -48,7 +48,7 @@ def _gpu(t, window, num_splits=0):
 
 
 @pytest.mark.parametrize("Q", [2, 3, 5, 9])
-@pytest.mark.parametrize("window,splits", [(0, 1), (0, 3), (100, 0), (1000, 2)])
+@pytest.mark.parametrize("window,splits", [(0, 1), (0, 3), (100, 0), (1000, 2), (0, 9), (0, 33)])
 def test_decode_mq_matches_oracle(oracle_mod, Q, window, splits):
     need_gpu()
     # lengths from exactly Q (every key is a draft token) to several blocks,

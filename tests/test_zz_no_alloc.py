@@ -125,24 +125,25 @@ def test_static_scratch_lowers_the_automatic_split_count(oracle_mod):
         assert_parity(out, ref, f"lowered static decode, call {call}")
 
 
-@pytest.mark.parametrize("q_len", [1, 3])
-def test_static_scratch_rows_that_cannot_be_computed_read_nan(q_len):
+@pytest.mark.parametrize("q_len,splits", [(1, 4), (3, 4), (1, 16), (3, 16)])
+def test_static_scratch_rows_that_cannot_be_computed_read_nan(q_len, splits):
     """A call whose sequence 1 has a length outside [q_len, max_blocks*128]
     reports BAD_LENGTH and writes NaN for that sequence's rows (never the
     previous call's partials, which are still in the array); the other
-    sequences' rows equal those of a valid call."""
+    sequences' rows equal those of a valid call.  4 splits merge with one
+    warp per row, 16 with four."""
     need_gpu()
     spec = scaled(WORKLOADS["decode_swa_s64"], S=4, L_min=5000, L_max=9000, window=0,
                   n_new=q_len, seed=23)
     t = make_decode(spec, device="cuda")
     first = torch.empty_like(t["q"])
-    _static_c(t, 0, first, 4)   # fills the array with this call's partials
+    _static_c(t, 0, first, splits)   # fills the array with this call's partials
     bad = dict(t)
     bad["seq_lens"] = t["seq_lens"].clone()
     bad["seq_lens"][1] = t["block_table"].shape[1] * 128 + 1
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = torch.zeros_like(t["q"])
-    _static_c(bad, 0, out, 4, status=status)
+    _static_c(bad, 0, out, splits, status=status)
     torch.cuda.synchronize()
     assert status.item() & binding.STATUS_BAD_LENGTH
     assert torch.isnan(out[1].float()).all()
