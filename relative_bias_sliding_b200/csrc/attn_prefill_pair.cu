@@ -299,9 +299,14 @@ attn_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const uint32_t ph1 = ((it + 1) / kPS) & 1;
                     if (!mbar_wait_cluster(&bar[V_READY + st], (it / kPS) & 1, abort_flag, a.status))
                         break;
-                    tc_fence_after();
                     const bool has_next = n < uhi;
-                    bool got_next = false;
+                    // the next tile's converted keys, checked before waiting for
+                    // P (they are normally ready long before): the wait then stays
+                    // off the P -> P.V -> QK^T -> S chain
+                    bool got_next = has_next && mbar_wait_cluster(&bar[K_READY + st1], ph1, abort_flag,
+                                                                  a.status);
+                    if (has_next && !got_next) break;
+                    tc_fence_after();
                     for (int t = 0; t < 2 && alive; ++t) {
                         if (in_range(t, n)) {
                             if (!mbar_wait_cluster(&bar[P_FULL + t], (n - lo[t]) & 1, abort_flag,
