@@ -53,7 +53,6 @@ MEASURED_TRAFFIC = {
     "prefill_swa_b4_t8192": 677_865_728 + 501_716_480,
     "prefill_paged_swa_b4_t8192": 677_026_816 + 497_247_232,
     "decode_swa_s64": 1_080_856_064 + 4_138_752,
-    "decode_mtp9_swa_s64": 1_089_919_744 + 8_944_640,
 }
 
 
@@ -256,9 +255,11 @@ class DecodeStep:
     def run_attn(self, stream=None):
         import relative_bias_sliding_b200 as ink
         t = self.t
+        # num_splits 0: the library's own plan, with the workspace sized for
+        # the split count it reports
         ink.attn_decode(t["q"], t["k_cache"], t["v_cache"], t["block_table"], t["seq_lens"],
                         t["bias"], window=self.spec.window, out=self.out, workspace=self.ws,
-                        num_splits=self.splits, stream=stream)
+                        num_splits=0, stream=stream)
 
     def run(self, stream=None):
         self.run_append(stream)
@@ -409,7 +410,7 @@ def e2e_decode(step, steps, stream):
                      t["k_cache"], t["v_cache"], d["block_table"], d["seq_lens"], stream=s)
         ink.attn_decode(d["q"], t["k_cache"], t["v_cache"], d["block_table"], d["seq_lens"],
                         t["bias"], window=step.spec.window, out=outs[b], workspace=step.ws,
-                        num_splits=step.splits, stream=s)
+                        num_splits=0, stream=s)
 
     def d2h(b, s):
         with torch.cuda.stream(s):

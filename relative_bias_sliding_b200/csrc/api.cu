@@ -15,9 +15,10 @@ cudaError_t launch_attn_prefill(const inkling_prefill_params &p, const CUtensorM
 cudaError_t launch_sconv_out(const inkling_sconv_out_params &p, cudaStream_t stream);
 cudaError_t launch_sconv_out_sharded(const inkling_sconv_out_sharded_params &p,
                                      cudaStream_t stream);
-cudaError_t launch_attn_decode_mq(const inkling_decode_params &p, int splits, void *workspace,
-                                  const CUtensorMap &tm_q, const CUtensorMap &tm_k,
-                                  const CUtensorMap &tm_v, cudaStream_t stream);
+cudaError_t launch_attn_decode_mq(const inkling_decode_params &p, int splits, int s_whole,
+                                  void *workspace, const CUtensorMap &tm_q,
+                                  const CUtensorMap &tm_k, const CUtensorMap &tm_v,
+                                  cudaStream_t stream);
 cudaError_t launch_attn_prefill_paged(const inkling_prefill_paged_params &p, const CUtensorMap &tm_q,
                                       const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                                       cudaStream_t stream);
@@ -152,6 +153,56 @@ int decode_splits(const inkling_decode_params &p, int num_sms) {
         }
     }
     return (int)best;
+}
+
+// How a decode call runs: sequences [0, s_whole) unsplit, the others in
+// `splits` key-range pieces (s_whole == num_seqs: no partials).
+struct DecodePlan {
+    int splits, s_whole;
+};
+
+// For num_splits = 0 in multi-token decode, when the (sequence, kv head)
+// units fill the slots: the sequences that fill whole waves run unsplit and
+// the rest, which would leave most of a last wave idle, in c pieces (2..8,
+// at least ~512 keys each) whose partials the combine merges.  Cost model,
+// in units of one whole unit's time, fitted to B200 measurements: a wave of
+// pieces costs 1/c + 0.1 (a piece's setup, pipeline fill and partials), the
+// combine 0.05; the plan is taken when it is 10% under the unsplit last wave
+// (1).  Measured, 9 draft tokens, window 4096, against the unsplit plan:
+// 40 sequences 0.138 ms vs 0.204 (8 pieces); 48 sequences 0.163 vs 0.206
+// (3 pieces); 128 sequences 0.412 vs 0.424 (2 pieces); 64 sequences would
+// take 4 pieces at 0.225 vs 0.220, and the model keeps it unsplit.
+static DecodePlan decode_plan(const inkling_decode_params &p, int num_sms) {
+    const int sp = decode_splits(p, num_sms);
+    DecodePlan plan{sp, sp == 1 ? p.num_seqs : 0};
+    const long slots = 2L * num_sms;
+    const long units = (long)p.num_seqs * p.num_kv_heads;
+    if (p.num_splits > 0 || sp != 1 || p.q_len <= 1 || units < slots) return plan;
+    const int s_whole = (int)(((units / slots) * slots) / p.num_kv_heads);
+    const long rest = units - (long)s_whole * p.num_kv_heads;
+    if (rest <= 0 || s_whole >= p.num_seqs) return plan;
+    const long max_keys = (long)p.max_blocks * 128;
+    const long keys = p.window > 0 ? (p.window < max_keys ? p.window : max_keys) : max_keys;
+    const long cap = ((keys + 63) / 64 + 1) / 8;
+    double best = 0.9;  // the remainder's last wave, unsplit, costs 1
+    int best_c = 1;
+    for (int c = 2; c <= 8 && c <= cap; ++c) {
+        const long waves = (rest * c + slots - 1) / slots;
+        const double t = (double)waves * (1.0 / c + 0.1) + 0.05;
+        if (t < best) {
+            best = t;
+            best_c = c;
+        }
+    }
+    if (best_c > 1) plan = DecodePlan{best_c, s_whole};
+    return plan;
+}
+
+// bytes of partials a plan needs (0: none)
+static size_t plan_workspace(const inkling_decode_params &p, const DecodePlan &plan) {
+    if (plan.splits <= 1 || plan.s_whole >= p.num_seqs) return 0;
+    const int32_t rows = (p.num_seqs - plan.s_whole) * (p.q_len > 1 ? p.q_len : 1);
+    return inkling_attn_decode_workspace_bytes(rows, p.num_q_heads, plan.splits);
 }
 
 inkling_status validate_decode(const inkling_decode_params *p) {
@@ -437,11 +488,11 @@ int32_t inkling_attn_decode_num_splits(const inkling_decode_params *p) {
     if (validate_decode(p) != INKLING_OK) return 0;
     int sms = 0;
     if (check_device(&sms) != INKLING_OK) return 0;
-    return decode_splits(*p, sms);
+    return decode_plan(*p, sms).splits;
 }
 
-static inkling_status decode_with(const inkling_decode_params *p, int splits, void *workspace,
-                                  size_t workspace_bytes, inkling_stream_t stream);
+static inkling_status decode_with(const inkling_decode_params *p, const DecodePlan &plan,
+                                  void *workspace, size_t workspace_bytes, inkling_stream_t stream);
 
 inkling_status inkling_attn_decode(const inkling_decode_params *p, void *workspace,
                                    size_t workspace_bytes, inkling_stream_t stream) {
@@ -451,7 +502,13 @@ inkling_status inkling_attn_decode(const inkling_decode_params *p, void *workspa
     if (p->num_seqs == 0) return INKLING_OK;
     int sms = 0;
     if ((st = check_device(&sms)) != INKLING_OK) return st;
-    return decode_with(p, decode_splits(*p, sms), workspace, workspace_bytes, stream);
+    DecodePlan plan = decode_plan(*p, sms);
+    // a split plan chosen automatically over a workspace too small for it
+    // (sized for one split) runs unsplit instead
+    if (p->num_splits == 0 && plan.s_whole > 0 && plan.s_whole < p->num_seqs &&
+        (!workspace || workspace_bytes < plan_workspace(*p, plan)))
+        plan = DecodePlan{1, p->num_seqs};
+    return decode_with(p, plan, workspace, workspace_bytes, stream);
 }
 
 inkling_status inkling_attn_decode_static(const inkling_decode_params *p, inkling_stream_t stream) {
@@ -465,7 +522,13 @@ inkling_status inkling_attn_decode_static(const inkling_decode_params *p, inklin
     size_t cap = 0;
     cudaError_t e = decode_static_scratch(&scratch, &cap);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the decode scratch");
-    int splits = decode_splits(*p, sms);
+    DecodePlan plan = decode_plan(*p, sms);
+    if (plan.s_whole > 0 && plan.s_whole < p->num_seqs) {
+        // whole + pieces: run it when its partials fit, else unsplit
+        if (plan_workspace(*p, plan) > cap) plan = DecodePlan{1, p->num_seqs};
+        return decode_with(p, plan, scratch, cap, stream);
+    }
+    int splits = plan.splits;
     const int32_t rows = decode_rows(*p);
     if (inkling_attn_decode_workspace_bytes(rows, p->num_q_heads, splits) > cap) {
         if (p->num_splits > 0)
@@ -478,12 +541,13 @@ inkling_status inkling_attn_decode_static(const inkling_decode_params *p, inklin
         while (splits > 1 && inkling_attn_decode_workspace_bytes(rows, p->num_q_heads, splits) > cap)
             --splits;
     }
-    return decode_with(p, splits, scratch, cap, stream);
+    return decode_with(p, DecodePlan{splits, splits == 1 ? p->num_seqs : 0}, scratch, cap, stream);
 }
 
-static inkling_status decode_with(const inkling_decode_params *p, int splits, void *workspace,
-                                  size_t workspace_bytes, inkling_stream_t stream) {
+static inkling_status decode_with(const inkling_decode_params *p, const DecodePlan &plan,
+                                  void *workspace, size_t workspace_bytes, inkling_stream_t stream) {
     inkling_status st;
+    const int splits = plan.splits;
     // one thread block per (sequence, kv head, split): the grid must fit a
     // signed 32-bit count
     if ((long)p->num_seqs * p->num_kv_heads * splits >= (1L << 31))
@@ -494,7 +558,7 @@ static inkling_status decode_with(const inkling_decode_params *p, int splits, vo
         if ((long)decode_rows(*p) * p->num_q_heads >= (1L << 31))
             return fail(INKLING_ERR_UNSUPPORTED, "%ld output rows to combine exceed 2^31",
                         (long)decode_rows(*p) * p->num_q_heads);
-        const size_t need = inkling_attn_decode_workspace_bytes(decode_rows(*p), p->num_q_heads, splits);
+        const size_t need = plan_workspace(*p, plan);
         if (!workspace || workspace_bytes < need)
             return fail(INKLING_ERR_INVALID, "workspace of %zu bytes given, %zu needed for %d splits",
                         workspace_bytes, need, splits);
@@ -518,8 +582,8 @@ static inkling_status decode_with(const inkling_decode_params *p, int splits, vo
         cuuint64_t qs[2] = {256, Hq * 256};
         cuuint32_t qb[3] = {64, (cuuint32_t)G, (cuuint32_t)p->q_len};
         if ((st = make_map(&tm_q, p->q, 3, qd, qs, qb)) != INKLING_OK) return st;
-        cudaError_t e = launch_attn_decode_mq(*p, splits, workspace, tm_q, tm_k, tm_v,
-                                              (cudaStream_t)stream);
+        cudaError_t e = launch_attn_decode_mq(*p, splits, plan.s_whole, workspace, tm_q, tm_k,
+                                              tm_v, (cudaStream_t)stream);
         if (e != cudaSuccess) return cuda_fail(e, "attn_decode (multi-token) launch");
         return INKLING_OK;
     }

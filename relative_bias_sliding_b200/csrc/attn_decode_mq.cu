@@ -39,7 +39,7 @@ cudaError_t launch_decode_combine(const float *part_o, const float *part_ml, uin
 // range, or a bounded wait gave up) reads NaN in out and lse; with splits, a
 // NaN partial makes the merged row NaN.
 __device__ __noinline__ void decode_nan_row(uint16_t *out, float *lse, float *part_ml, int splits,
-                                            long pair, int split) {
+                                            long pair, long pbase, int split) {
     const float nanv = __int_as_float(0x7fc00000);
     if (splits == 1) {
         const uint32_t nb = 0x7fc07fc0u;
@@ -47,7 +47,7 @@ __device__ __noinline__ void decode_nan_row(uint16_t *out, float *lse, float *pa
         for (int c = 0; c < 16; ++c) dst[c] = make_uint4(nb, nb, nb, nb);
         if (lse) lse[pair] = nanv;
     } else {
-        const long pi = pair * splits + split;
+        const long pi = (pair - pbase) * splits + split;
         part_ml[pi * 2] = nanv;
         part_ml[pi * 2 + 1] = nanv;
     }
@@ -90,6 +90,11 @@ struct DecodeMqArgs {
     float *part_o, *part_ml;
     int32_t *status;
     int S, Q, Hq, Hkv, G, max_blocks, num_blocks, window, d_max, splits;
+    // sequences [0, s_whole) run unsplit (one block per kv head, output
+    // written directly); sequences [s_whole, S) in `splits` key-range pieces
+    // whose partials start at row pbase = s_whole * Q * Hq
+    int s_whole;
+    long pbase;
 };
 
 __global__ void __launch_bounds__(192, 2)
@@ -103,9 +108,22 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int s = blockIdx.x % a.S;
-    const int kvh = (blockIdx.x / a.S) % a.Hkv;
-    const int split = blockIdx.x / (a.S * a.Hkv);
+    // blocks of the whole sequences first (they are dispatched first), then
+    // the pieces of the others
+    const int nwhole = a.s_whole * a.Hkv;
+    int s, kvh, split, splits;
+    if ((int)blockIdx.x < nwhole) {
+        s = blockIdx.x % a.s_whole;
+        kvh = blockIdx.x / a.s_whole;
+        split = 0;
+        splits = 1;
+    } else {
+        const int j = blockIdx.x - nwhole, Sr = a.S - a.s_whole;
+        s = a.s_whole + j % Sr;
+        kvh = (j / Sr) % a.Hkv;
+        split = j / (Sr * a.Hkv);
+        splits = a.splits;
+    }
     const int Q = a.Q, G = a.G, rows = G * Q;
 
     // key tiles of this sequence (union of its rows' windows) and this split
@@ -115,7 +133,7 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     int ta = 0, tb = 0;
     if (!bad_len) {
         const int t_lo = klo / kMqTile, t_hi = (L - 1) / kMqTile;
-        const int per = (t_hi - t_lo + a.splits) / a.splits;
+        const int per = (t_hi - t_lo + splits) / splits;
         ta = min(t_hi + 1, t_lo + split * per);
         tb = min(t_hi + 1, ta + per);
     } else if (threadIdx.x == 0 && split == 0 && kvh == 0) {
@@ -324,7 +342,7 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         auto o = [&](int i) { return __uint_as_float(ob[i]); };
         if (rv && !bad_len && !*abort_flag) {
             const long pair = ((long)s * Q + qi) * a.Hq + h;
-            if (a.splits == 1) {
+            if (splits == 1) {
                 const float inv = (l > 0.f) ? 1.f / l : 0.f;
                 uint4 *dst = (uint4 *)(a.out + pair * 128);
 #pragma unroll
@@ -338,7 +356,7 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
                 if (a.lse) a.lse[pair] = (l > 0.f) ? m_ref + __logf(l) : -INFINITY;
             } else {
-                const long pi = pair * a.splits + split;
+                const long pi = (pair - a.pbase) * splits + split;
                 float4 *po = (float4 *)(a.part_o + pi * 128);
                 if (have_o) {
 #pragma unroll
@@ -463,13 +481,17 @@ decode_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // that the main loop's code stays as it is without this rare path (in the
     // epilogue it cost the kernel 6%)
     if (warp < 4 && (int)threadIdx.x < rows && (bad_len || *abort_flag))
-        decode_nan_row(a.out, a.lse, a.part_ml, a.splits,
-                       ((long)s * Q + threadIdx.x / G) * a.Hq + kvh * G + threadIdx.x % G, split);
+        decode_nan_row(a.out, a.lse, a.part_ml, splits,
+                       ((long)s * Q + threadIdx.x / G) * a.Hq + kvh * G + threadIdx.x % G, a.pbase,
+                       split);
 }
 
-cudaError_t launch_attn_decode_mq(const inkling_decode_params &p, int splits, void *workspace,
-                                  const CUtensorMap &tm_q, const CUtensorMap &tm_k,
-                                  const CUtensorMap &tm_v, cudaStream_t stream) {
+// s_whole: sequences [0, s_whole) run unsplit, the rest in `splits` pieces
+// (s_whole == num_seqs: no partials; 0: every sequence split).
+cudaError_t launch_attn_decode_mq(const inkling_decode_params &p, int splits, int s_whole,
+                                  void *workspace, const CUtensorMap &tm_q,
+                                  const CUtensorMap &tm_k, const CUtensorMap &tm_v,
+                                  cudaStream_t stream) {
     DecodeMqArgs a;
     a.block_table = p.block_table;
     a.seq_lens = p.seq_lens;
@@ -486,18 +508,24 @@ cudaError_t launch_attn_decode_mq(const inkling_decode_params &p, int splits, vo
     a.num_blocks = p.num_blocks;
     a.window = p.window;
     a.d_max = p.d_max;
+    if (splits == 1) s_whole = p.num_seqs;
     a.splits = splits;
-    const long rows_total = (long)p.num_seqs * p.q_len * p.num_q_heads;
+    a.s_whole = s_whole;
+    a.pbase = (long)s_whole * p.q_len * p.num_q_heads;
+    const long rows_part = (long)(p.num_seqs - s_whole) * p.q_len * p.num_q_heads;
     a.part_o = (float *)workspace;
-    a.part_ml = splits > 1 ? (float *)workspace + rows_total * splits * 128 : nullptr;
+    a.part_ml = rows_part > 0 ? (float *)workspace + rows_part * splits * 128 : nullptr;
     cudaError_t e = cudaFuncSetAttribute(decode_mq_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kMqSmem);
     if (e != cudaSuccess) return e;
-    const long grid = (long)p.num_seqs * p.num_kv_heads * splits;
+    const long grid = (long)s_whole * p.num_kv_heads +
+                      (long)(p.num_seqs - s_whole) * p.num_kv_heads * splits;
+    if (grid == 0) return cudaSuccess;
     decode_mq_tc_kernel<<<(unsigned)grid, 192, kMqSmem, stream>>>(tm_q, tm_k, tm_v, a);
     e = cudaGetLastError();
-    if (e != cudaSuccess || splits == 1) return e;
-    return launch_decode_combine(a.part_o, a.part_ml, a.out, a.lse, rows_total, splits, stream);
+    if (e != cudaSuccess || rows_part == 0) return e;
+    return launch_decode_combine(a.part_o, a.part_ml, a.out + a.pbase * 128,
+                                 a.lse ? a.lse + a.pbase : nullptr, rows_part, splits, stream);
 }
 
 }  // namespace inkling

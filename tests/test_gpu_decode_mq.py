@@ -138,6 +138,52 @@ def test_decode_mq_static_matches_workspace_call():
     assert torch.equal(a, b)
 
 
+def test_decode_mq_whole_and_split_sequences_match_oracle(oracle_mod):
+    """48 sequences x 8 kv heads fill the SMs' slots: the automatic plan runs
+    the sequences that fill whole waves unsplit and the rest in key-range
+    pieces merged by the combine (reported split count > 1).  Every row and
+    lse against the oracle."""
+    need_gpu()
+    S, Q = 48, 3
+    rng = np.random.default_rng(5)
+    lens = [int(x) for x in rng.integers(Q, 1500, size=S)]
+    t = _inputs(S, Q, lens, Hq=64, Hkv=8, d_max=1024, seed=55)
+    dev = {k: v.cuda() for k, v in t.items()}
+    reported = ink.decode_num_splits(dev["q"], dev["k_cache"], dev["v_cache"], dev["block_table"],
+                                     dev["seq_lens"], dev["bias"], window=0)
+    assert reported > 1, "the case must take the whole + pieces plan"
+    ref, ref_lse = _oracle(oracle_mod, t, 0)
+    out, lse = _gpu(t, 0)
+    assert_parity(out, ref, "whole + pieces plan")
+    np.testing.assert_allclose(lse.cpu().numpy().reshape(-1), ref_lse, rtol=0, atol=2e-3)
+    # the same call with one split (no partials) agrees with it closely
+    one, _ = _gpu(t, 0, 1)
+    assert (one.float() - out.float()).abs().max().item() < 1e-2
+
+
+def test_decode_mq_whole_and_split_bad_length_rows_read_nan():
+    """With the whole + pieces plan, a sequence of bad length among the whole
+    ones and one among the split ones both read NaN; the others are those of
+    a valid call."""
+    need_gpu()
+    S, Q = 48, 2
+    rng = np.random.default_rng(6)
+    lens = [int(x) for x in rng.integers(Q, 900, size=S)]
+    t = _inputs(S, Q, lens, Hq=64, Hkv=8, d_max=1024, seed=56)
+    good, _ = _gpu(t, 0)
+    bad = dict(t)
+    bad["seq_lens"] = t["seq_lens"].clone()
+    bad["seq_lens"][0] = 1           # a whole sequence: fewer than q_len tokens
+    bad["seq_lens"][S - 1] = 1       # a split sequence
+    dev = {k: v.cuda() for k, v in bad.items()}
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = ink.attn_decode(**dev, window=0, status=status)
+    torch.cuda.synchronize()
+    assert status.item() & 4   # INKLING_STATUS_BAD_LENGTH
+    assert torch.isnan(out[0].float()).all() and torch.isnan(out[S - 1].float()).all()
+    assert torch.equal(out[1:S - 1], good[1:S - 1])
+
+
 def test_decode_mq_rejects_too_many_rows():
     need_gpu()
     t = _inputs(1, 11, [100], Hq=16, Hkv=2, d_max=64)   # G 8 x 11 tokens = 88 rows
