@@ -360,10 +360,10 @@ size_t inkling_attn_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads
 
 /* The split count to size the workspace for (resolves num_splits = 0);
  * returns 0 for invalid parameters.  With num_splits = 0 it is the count the
- * call uses: for every sequence, or, in multi-token decode whose (sequence,
- * kv head) units fill the SMs, for the sequences past those that fill whole
- * waves (those run unsplit).  A call with num_splits = 0 whose workspace is
- * smaller than that count needs runs every sequence unsplit instead. */
+ * call uses: for every sequence, or, when the (sequence, kv head) units fill
+ * the SMs, for the sequences past those that fill whole waves (those run
+ * unsplit).  A call with num_splits = 0 whose workspace is smaller than that
+ * count needs runs every sequence unsplit instead. */
 int32_t inkling_attn_decode_num_splits(const inkling_decode_params *p);
 
 /* workspace: device, >= inkling_attn_decode_workspace_bytes(...) bytes, 16-byte

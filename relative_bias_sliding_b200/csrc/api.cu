@@ -24,8 +24,8 @@ cudaError_t launch_attn_prefill_paged(const inkling_prefill_paged_params &p, con
                                       cudaStream_t stream);
 cudaError_t launch_attn_prefill_pair(const inkling_prefill_params &p, const CUtensorMap *maps,
                                      cudaStream_t stream);
-cudaError_t launch_attn_decode(const inkling_decode_params &p, int splits, void *workspace,
-                               const CUtensorMap &tm_k, const CUtensorMap &tm_v,
+cudaError_t launch_attn_decode(const inkling_decode_params &p, int splits, int s_whole,
+                               void *workspace, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                                cudaStream_t stream);
 cudaError_t decode_static_scratch(void **ptr, size_t *bytes);
 cudaError_t launch_wait_timeout_probe(int32_t *status, uint32_t limit_us, cudaStream_t stream);
@@ -161,23 +161,25 @@ struct DecodePlan {
     int splits, s_whole;
 };
 
-// For num_splits = 0 in multi-token decode, when the (sequence, kv head)
-// units fill the slots: the sequences that fill whole waves run unsplit and
-// the rest, which would leave most of a last wave idle, in c pieces (2..8,
-// at least ~512 keys each) whose partials the combine merges.  Cost model,
-// in units of one whole unit's time, fitted to B200 measurements: a wave of
-// pieces costs 1/c + 0.1 (a piece's setup, pipeline fill and partials), the
-// combine 0.05; the plan is taken when it is 10% under the unsplit last wave
-// (1).  Measured, 9 draft tokens, window 4096, against the unsplit plan:
-// 40 sequences 0.138 ms vs 0.204 (8 pieces); 48 sequences 0.163 vs 0.206
-// (3 pieces); 128 sequences 0.412 vs 0.424 (2 pieces); 64 sequences would
-// take 4 pieces at 0.225 vs 0.220, and the model keeps it unsplit.
+// For num_splits = 0, when the (sequence, kv head) units fill the slots: the
+// sequences that fill whole waves run unsplit and the rest, which would leave
+// most of a last wave idle, in c pieces (2..8, at least ~512 keys each) whose
+// partials the combine merges.  Cost model, in units of one whole unit's
+// time, fitted to B200 measurements: a wave of pieces costs 1/c + 0.1 (a
+// piece's setup, pipeline fill and partials), the combine 0.05; the plan is
+// taken when it is 10% under the unsplit last wave (1).  Measured against the
+// unsplit plan (window 4096, KV TB/s):
+//   1 token:   40 sequences 4.34 -> 5.70 (8 pieces), 48: 5.20 -> 5.91 (3),
+//              80: 5.43 -> 6.22 (6), 128: 6.20 -> 6.38 (2);
+//   9 tokens:  40 sequences 3.15 -> 4.70 (8), 48: 3.76 -> 4.82 (3),
+//              80: 4.23 -> 4.97 (6), 128: 4.94 -> 5.09 (2);
+//   64 sequences stay unsplit (9 tokens in 4 pieces measured 4.71 vs 4.87).
 static DecodePlan decode_plan(const inkling_decode_params &p, int num_sms) {
     const int sp = decode_splits(p, num_sms);
     DecodePlan plan{sp, sp == 1 ? p.num_seqs : 0};
     const long slots = 2L * num_sms;
     const long units = (long)p.num_seqs * p.num_kv_heads;
-    if (p.num_splits > 0 || sp != 1 || p.q_len <= 1 || units < slots) return plan;
+    if (p.num_splits > 0 || sp != 1 || units < slots) return plan;
     const int s_whole = (int)(((units / slots) * slots) / p.num_kv_heads);
     const long rest = units - (long)s_whole * p.num_kv_heads;
     if (rest <= 0 || s_whole >= p.num_seqs) return plan;
@@ -590,7 +592,8 @@ static inkling_status decode_with(const inkling_decode_params *p, const DecodePl
     cuuint32_t box[2] = {64, 64};
     if ((st = make_map(&tm_k, p->k_cache, 2, dims, str, box)) != INKLING_OK) return st;
     if ((st = make_map(&tm_v, p->v_cache, 2, dims, str, box)) != INKLING_OK) return st;
-    cudaError_t e = launch_attn_decode(*p, splits, workspace, tm_k, tm_v, (cudaStream_t)stream);
+    cudaError_t e = launch_attn_decode(*p, splits, plan.s_whole, workspace, tm_k, tm_v,
+                                       (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "attn_decode launch");
     return INKLING_OK;
 }

@@ -41,6 +41,11 @@ struct DecodeArgs {
     float *part_ml;  // [S, Hq, splits, 2] (max in log2 units, sum)
     int32_t *status;
     int S, Hq, Hkv, G, max_blocks, num_blocks, window, d_max, splits;
+    // sequences [0, s_whole) run unsplit (output written directly); sequences
+    // [s_whole, S) in `splits` key-range pieces whose partials start at row
+    // pbase = s_whole * Hq
+    int s_whole;
+    long pbase;
 };
 
 INK_DEV void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
@@ -75,9 +80,22 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
     volatile int *abort_flag = (volatile int *)(empty + kDecStages);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int s = blockIdx.x % a.S;
-    const int kvh = (blockIdx.x / a.S) % a.Hkv;
-    const int split = blockIdx.x / (a.S * a.Hkv);
+    // blocks of the whole sequences first (they are dispatched first), then
+    // the pieces of the others
+    const int nwhole = a.s_whole * a.Hkv;
+    int s, kvh, split, splits;
+    if ((int)blockIdx.x < nwhole) {
+        s = blockIdx.x % a.s_whole;
+        kvh = blockIdx.x / a.s_whole;
+        split = 0;
+        splits = 1;
+    } else {
+        const int j = blockIdx.x - nwhole, Sr = a.S - a.s_whole;
+        s = a.s_whole + j % Sr;
+        kvh = (j / Sr) % a.Hkv;
+        split = j / (Sr * a.Hkv);
+        splits = a.splits;
+    }
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kDecStages; ++i) {
@@ -96,7 +114,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
     int ca = 0, cb = 0;
     if (!bad_len) {
         const int c_lo = lo >> 6, c_hi = (L + 63) >> 6;
-        const int per = (c_hi - c_lo + a.splits - 1) / a.splits;
+        const int per = (c_hi - c_lo + splits - 1) / splits;
         ca = min(c_hi, c_lo + split * per);
         cb = min(c_hi, ca + per);
     } else if (threadIdx.x == 0 && split == 0 && kvh == 0) {
@@ -274,12 +292,12 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
             // result; with splits the NaN partial makes the merged row NaN
             const float nanv = __int_as_float(0x7fc00000);
             const int hh = kvh * a.G + gg;
-            if (a.splits == 1) {
+            if (splits == 1) {
                 const uint32_t nb = 0x7fc07fc0u;
                 *(uint4 *)(a.out + ((long)s * a.Hq + hh) * 128 + d0) = make_uint4(nb, nb, nb, nb);
                 if (a.lse && (u & 15) == 0) a.lse[(long)s * a.Hq + hh] = nanv;
             } else if ((u & 15) == 0) {
-                const long pi = ((long)s * a.Hq + hh) * a.splits + split;
+                const long pi = ((long)s * a.Hq + hh - a.pbase) * splits + split;
                 a.part_ml[pi * 2] = nanv;
                 a.part_ml[pi * 2 + 1] = nanv;
             }
@@ -303,7 +321,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
                 acc[e] = v;
             }
             const int hh = kvh * a.G + gg;
-            if (a.splits == 1) {
+            if (splits == 1) {
                 const float inv = (Ls > 0.f) ? 1.f / Ls : 0.f;
                 uint4 pk;
                 pk.x = pack_bf16(acc[0] * inv, acc[1] * inv);
@@ -315,7 +333,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
                     a.lse[(long)s * a.Hq + hh] =
                         (Ls > 0.f) ? (M + __log2f(Ls)) * 0.6931471805599453f : -INFINITY;
             } else {
-                const long pi = ((long)s * a.Hq + hh) * a.splits + split;
+                const long pi = ((long)s * a.Hq + hh - a.pbase) * splits + split;
                 float4 *po = (float4 *)(a.part_o + pi * 128 + d0);
                 po[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
                 po[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
@@ -430,8 +448,10 @@ cudaError_t launch_decode_combine(const float *part_o, const float *part_ml, uin
     return launch_combine_wpr<1>(part_o, part_ml, out, lse, rows, splits, stream);
 }
 
-cudaError_t launch_attn_decode(const inkling_decode_params &p, int splits, void *workspace,
-                               const CUtensorMap &tm_k, const CUtensorMap &tm_v,
+// s_whole: sequences [0, s_whole) run unsplit, the rest in `splits` pieces
+// (s_whole == num_seqs: no partials; 0: every sequence split).
+cudaError_t launch_attn_decode(const inkling_decode_params &p, int splits, int s_whole,
+                               void *workspace, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                                cudaStream_t stream) {
     DecodeArgs a;
     a.q = (const uint16_t *)p.q;
@@ -440,7 +460,6 @@ cudaError_t launch_attn_decode(const inkling_decode_params &p, int splits, void 
     a.bias = p.bias;
     a.out = (uint16_t *)p.out;
     a.lse = p.lse;
-    const long pairs = (long)p.num_seqs * p.num_q_heads;
     a.part_o = (float *)workspace;
     a.status = p.status;
     a.S = p.num_seqs;
@@ -451,17 +470,23 @@ cudaError_t launch_attn_decode(const inkling_decode_params &p, int splits, void 
     a.num_blocks = p.num_blocks;
     a.window = p.window;
     a.d_max = p.d_max;
+    if (splits == 1) s_whole = p.num_seqs;
     a.splits = splits;
-    const long rows_total = pairs;
-    a.part_ml = splits > 1 ? (float *)workspace + rows_total * splits * 128 : nullptr;
-    const long grid = (long)p.num_seqs * p.num_kv_heads * splits;
+    a.s_whole = s_whole;
+    a.pbase = (long)s_whole * p.num_q_heads;
+    const long rows_part = (long)(p.num_seqs - s_whole) * p.num_q_heads;
+    a.part_ml = rows_part > 0 ? (float *)workspace + rows_part * splits * 128 : nullptr;
+    const long grid = (long)s_whole * p.num_kv_heads +
+                      (long)(p.num_seqs - s_whole) * p.num_kv_heads * splits;
+    if (grid == 0) return cudaSuccess;
     cudaError_t e0 = cudaFuncSetAttribute(decode_split_kernel,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
     if (e0 != cudaSuccess) return e0;
     decode_split_kernel<<<(unsigned)grid, 160, kDecSmem, stream>>>(tm_k, tm_v, a);
     cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess || splits == 1) return e;
-    return launch_decode_combine(a.part_o, a.part_ml, a.out, a.lse, rows_total, splits, stream);
+    if (e != cudaSuccess || rows_part == 0) return e;
+    return launch_decode_combine(a.part_o, a.part_ml, a.out + a.pbase * 128,
+                                 a.lse ? a.lse + a.pbase : nullptr, rows_part, splits, stream);
 }
 
 // ---------------------------------------------------------------------------

@@ -88,6 +88,38 @@ def test_decode_block_permutation_is_bit_exact():
     assert torch.equal(out1, out2)
 
 
+def test_decode_whole_and_split_sequences_match_oracle(oracle_mod):
+    """48 sequences x 8 kv heads fill the SMs' slots: the automatic plan runs
+    the sequences that fill whole waves unsplit and the rest in key-range
+    pieces merged by the combine (reported split count > 1).  Every (seq,
+    head) row and lse against the oracle; a sequence of bad length among the
+    whole ones and one among the split ones read NaN."""
+    need_gpu()
+    S = 48
+    rng = np.random.default_rng(8)
+    lens = [int(x) for x in rng.integers(1, 3000, size=S)]
+    t, W = _inputs(S, lens, Hq=64, Hkv=8, window=0, d_max=2048, seed=58)
+    dev = {k: v.cuda() for k, v in t.items()}
+    reported = ink.decode_num_splits(dev["q"], dev["k_cache"], dev["v_cache"], dev["block_table"],
+                                     dev["seq_lens"], dev["bias"], window=0)
+    assert reported > 1, "the case must take the whole + pieces plan"
+    ref, ref_lse = _oracle(oracle_mod, t, W)
+    out, lse = _gpu(t, W)
+    assert_parity(out, ref, "whole + pieces plan")
+    np.testing.assert_allclose(lse.cpu().numpy().reshape(-1), ref_lse, rtol=0, atol=2e-3)
+    bad = dict(t)
+    bad["seq_lens"] = t["seq_lens"].clone()
+    bad["seq_lens"][0] = 0
+    bad["seq_lens"][S - 1] = 0
+    bdev = {k: v.cuda() for k, v in bad.items()}
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out2 = ink.attn_decode(**bdev, window=0, status=status)
+    torch.cuda.synchronize()
+    assert status.item() & 4   # INKLING_STATUS_BAD_LENGTH
+    assert torch.isnan(out2[0].float()).all() and torch.isnan(out2[S - 1].float()).all()
+    assert torch.equal(out2[1:S - 1], out[1:S - 1])
+
+
 @pytest.mark.parametrize("splits", [8, 12, 20, 40])
 def test_decode_combine_warps_per_row_matches_oracle(oracle_mod, splits):
     """The combine merges each row with 1, 2, 4 or 8 warps by split count:
