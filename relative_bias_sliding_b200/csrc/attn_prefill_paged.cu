@@ -232,9 +232,14 @@ attn_prefill_paged_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const int st = it & 1, st1 = (it + 1) & 1;
                     const uint32_t ph1 = ((it + 1) >> 1) & 1;
                     if (!mbar_wait(&bar[G_VFULL + st], (it >> 1) & 1, abort_flag, a.status)) break;
-                    tc_fence_after();
                     const bool has_next = nt < uhi;
-                    bool got_next = false;
+                    // the next key tile, checked before waiting for P (it was
+                    // requested two tiles ago): the wait then stays off the
+                    // P -> P.V -> QK^T -> S chain
+                    bool got_next = has_next && mbar_wait(&bar[G_KFULL + st1], ph1, abort_flag,
+                                                          a.status);
+                    if (has_next && !got_next) break;
+                    tc_fence_after();
                     for (int t = 0; t < 2 && alive; ++t) {
                         if (in_range(t, nt)) {
                             if (!mbar_wait(&bar[G_PFULL + t], (nt - lo[t]) & 1, abort_flag,
