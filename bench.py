@@ -50,8 +50,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # 3 warm-up launches; profiles/ holds the summaries and commands).  Remove an
 # entry when its kernel changes until it is captured again.
 MEASURED_TRAFFIC = {
-    "prefill_swa_b4_t8192": 677_865_728 + 501_716_480,
-    "prefill_paged_swa_b4_t8192": 677_026_816 + 497_247_232,
+    "prefill_swa_b4_t8192": 680_339_712 + 501_876_992,
+    "prefill_paged_swa_b4_t8192": 677_535_232 + 496_792_064,
     "decode_swa_s64": 1_080_809_216 + 3_773_440,
     "decode_mtp9_swa_s64": 1_089_955_584 + 8_819_968,
 }
