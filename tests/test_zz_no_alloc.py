@@ -91,6 +91,33 @@ def test_static_scratch_decode_matches_oracle(oracle_mod, window):
         assert_parity(out, ref, f"static decode, window {window}, call {call}")
 
 
+def test_static_scratch_runs_the_whole_and_pieces_plan(oracle_mod):
+    """48 sequences x 3 draft tokens fill the SMs' slots: the automatic plan
+    runs the first sequences unsplit and the rest in pieces, and its partials
+    (a few MB) fit the library's array.  Two calls in a row equal
+    inkling_attn_decode with a workspace bit for bit, and the oracle on every
+    row."""
+    need_gpu()
+    spec = scaled(WORKLOADS["decode_swa_s64"], S=48, L_min=200, L_max=3000, window=1000,
+                  n_new=3, seed=24)
+    t = make_decode(spec, device="cuda")
+    assert ink.decode_num_splits(t["q"], t["k_cache"], t["v_cache"], t["block_table"],
+                                 t["seq_lens"], t["bias"], window=spec.window) > 1
+    ref_ws = ink.attn_decode(t["q"], t["k_cache"], t["v_cache"], t["block_table"],
+                             t["seq_lens"], t["bias"], window=spec.window)
+    host = {k: v.cpu() for k, v in t.items()}
+    ref, _ = oracle_mod.decode_mq_rows(u16(host["q"]), u16(host["k_cache"]),
+                                       u16(host["v_cache"]), host["block_table"].numpy(),
+                                       host["seq_lens"].numpy(), host["bias"].numpy(),
+                                       spec.window, spec.D_max)
+    for call in range(2):
+        out = torch.full_like(t["q"], float("nan"))
+        _static_c(t, spec.window, out, 0)
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref_ws), f"call {call}: differs from the workspace call"
+        assert_parity(out, ref, f"whole + pieces static decode, call {call}")
+
+
 def test_static_scratch_lowers_the_automatic_split_count(oracle_mod):
     """Multi-token decode (10 draft tokens) of 2 sequences of 40,000 tokens:
     the automatic split count needs more partials than the 8 MiB array holds,
