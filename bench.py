@@ -901,9 +901,9 @@ def main():
     if not args.no_e2e:
         e2e_parts = []
         if pre:
-            e2e_parts.append(("pre",) + e2e_prefill(pre, max(3, args.steps // 4), stream))
+            e2e_parts.append(("pre",) + e2e_prefill(pre, max(10, args.steps), stream))
         if dec:
-            e2e_parts.append(("dec",) + e2e_decode(dec, max(3, args.steps // 4), stream))
+            e2e_parts.append(("dec",) + e2e_decode(dec, max(10, args.steps), stream))
         e2e = e2e_parts
 
     line = {"metric": METRIC, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -938,7 +938,10 @@ def main():
         if pre:
             ms, h2d, d2h = parts["pre"]
             line["e2e"] = {"value": pre.flops / (ms * 1e-3) / 1e12 * world, "unit": "TFLOP/s",
-                           "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+                           "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                           "steps": max(10, args.steps),
+                           "pipelined": "copy-in, compute and copy-out of successive steps "
+                                        "overlap on three streams"}
             if dec:
                 ms2, h2d2, d2h2 = parts["dec"]
                 line["e2e"]["decode"] = {"value": dec.kv_bytes / (ms2 * 1e-3) / 1e9 * world,
