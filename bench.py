@@ -3,7 +3,10 @@
 
 One step = one pass of the whole hot path over one batch of synthetic input:
   * prefill: the sliding-window prefill workload (B=4, T=8192, Hq=64, Hkv=8,
-    d=128, window 4096) through inkling_attn_prefill (sconv fused);
+    d=128, window 4096) through inkling_attn_prefill on its automatic path
+    (at this length two kernels: the sconv of all keys/values written once
+    into a preallocated workspace in the paged layout, then the paged
+    prefill kernel; the fused one-kernel path is timed beside it);
   * decode: the sliding-window decode workload (64 sequences, lengths uniform
     in [1024, 32768], window 4096, paged 128-token blocks) through
     inkling_sconv_kv + inkling_attn_decode.
@@ -50,8 +53,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # 3 warm-up launches; profiles/ holds the summaries and commands).  Remove an
 # entry when its kernel changes until it is captured again.
 MEASURED_TRAFFIC = {
-    "prefill_swa_b4_t8192": 680_339_712 + 501_876_992,
-    "prefill_paged_swa_b4_t8192": 677_535_232 + 496_792_064,
+    "prefill_swa_b4_t8192": 677_133_312 + 499_282_176,   # paged kernel of the two-pass call
+    "prefill_swa_b4_t8192 fused": 680_339_712 + 501_876_992,
     "decode_swa_s64": 1_080_809_216 + 3_773_440,
     "decode_mtp9_swa_s64": 1_089_955_584 + 8_819_968,
 }
@@ -192,19 +195,68 @@ def hbm_roofline(achieved, kernel, traffic=None):
 # ----------------------------------------------------------- GPU workload --
 
 class PrefillStep:
+    """One prefill call on the automatic path (two-pass from 2048 tokens:
+    sconv into a preallocated workspace, then the paged prefill kernel; fused
+    below), plus the fused kernel and the cache-filling variants of the same
+    call, and the two passes as separate public calls for their timings."""
+
     def __init__(self, spec, device):
         import torch
+        import relative_bias_sliding_b200 as ink
         from relative_bias_sliding_b200.inputs import make_prefill
         self.spec = spec
         self.t = make_prefill(spec, device=device)
         self.out = torch.empty_like(self.t["q"])
         self.flops = spec.flops
+        nbytes = ink.prefill_workspace_bytes(spec.B, spec.T, spec.Hq, spec.Hkv)
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=device) if nbytes else None
+        self.two_pass = nbytes > 0
+        self.launches = 2 if self.two_pass else 1
+        self.path = "two_pass" if self.two_pass else "fused"
+        self.kernel = "attn_prefill_paged_kernel" if self.two_pass else "attn_prefill_pair_kernel"
 
     def run(self, stream=None):
         import relative_bias_sliding_b200 as ink
         t = self.t
         ink.attn_prefill(t["q"], t["k_raw"], t["v_raw"], t["w_k"], t["w_v"], t["bias"],
-                         window=self.spec.window, out=self.out, stream=stream)
+                         window=self.spec.window, out=self.out, stream=stream,
+                         workspace=self.ws)
+
+    def run_fused(self, stream=None):
+        import relative_bias_sliding_b200 as ink
+        t = self.t
+        ink.attn_prefill(t["q"], t["k_raw"], t["v_raw"], t["w_k"], t["w_v"], t["bias"],
+                         window=self.spec.window, out=self.out, stream=stream, path="fused")
+
+    def add_parts(self, device):
+        """Buffers for the two passes as separate public calls: the sconv
+        append of all T tokens into a cache in the scratch's block order
+        (sequence b on blocks b*nb ...), then the paged prefill of every
+        sequence as one chunk of T rows."""
+        import torch
+        B, T, Hq, Hkv = self.spec.B, self.spec.T, self.spec.Hq, self.spec.Hkv
+        nb = (T + 127) // 128
+        self.p_bt = torch.arange(B * nb, dtype=torch.int32, device=device).reshape(B, nb)
+        self.p_kc = torch.zeros((B * nb, Hkv, 128, 128), dtype=torch.bfloat16, device=device)
+        self.p_vc = torch.zeros_like(self.p_kc)
+        self.p_ks = torch.zeros((B, 3, Hkv * 128), dtype=torch.bfloat16, device=device)
+        self.p_vs = torch.zeros_like(self.p_ks)
+        self.p_lens = torch.full((B,), T, dtype=torch.int32, device=device)
+        self.p_cu = torch.arange(0, (B + 1) * T, T, dtype=torch.int32, device=device)
+
+    def run_part_sconv(self, stream=None):
+        import relative_bias_sliding_b200 as ink
+        t = self.t
+        ink.sconv_kv(t["k_raw"], t["v_raw"], t["w_k"], t["w_v"], self.p_ks, self.p_vs,
+                     self.p_kc, self.p_vc, self.p_bt, self.p_lens, stream=stream)
+
+    def run_part_attn(self, stream=None):
+        import relative_bias_sliding_b200 as ink
+        t, sp = self.t, self.spec
+        rows = sp.B * sp.T
+        ink.attn_prefill_paged(t["q"].view(rows, sp.Hq, sp.d), self.p_cu, self.p_kc, self.p_vc,
+                               self.p_bt, self.p_lens, t["bias"], window=sp.window, max_q=sp.T,
+                               out=self.out.view(rows, sp.Hq, sp.d), stream=stream)
 
     def add_cache(self, device):
         """Paged cache, block table and sconv states for the cache-filling
@@ -219,14 +271,16 @@ class PrefillStep:
         self.ks = torch.zeros((B, 3, Hkv * 128), dtype=torch.bfloat16, device=device)
         self.vs = torch.zeros_like(self.ks)
 
-    def run_fill(self, stream=None):
+    def run_fill(self, stream=None, path="auto"):
         import relative_bias_sliding_b200 as ink
         t = self.t
         ink.attn_prefill(t["q"], t["k_raw"], t["v_raw"], t["w_k"], t["w_v"], t["bias"],
                          window=self.spec.window, out=self.out, stream=stream, k_cache=self.kc,
-                         v_cache=self.vc, block_table=self.bt, k_state=self.ks, v_state=self.vs)
+                         v_cache=self.vc, block_table=self.bt, k_state=self.ks, v_state=self.vs,
+                         path=path)
 
-    launches = 1
+    def run_fill_fused(self, stream=None):
+        self.run_fill(stream, path="fused")
 
 
 class DecodeStep:
@@ -375,7 +429,8 @@ def e2e_prefill(step, steps, stream):
 
     def compute(b, s):
         ink.attn_prefill(dev[b]["q"], dev[b]["k_raw"], dev[b]["v_raw"], t["w_k"], t["w_v"],
-                         t["bias"], window=step.spec.window, out=outs[b], stream=s)
+                         t["bias"], window=step.spec.window, out=outs[b], stream=s,
+                         workspace=step.ws)  # the calls run in order on one stream
 
     def d2h(b, s):
         with torch.cuda.stream(s):
@@ -824,15 +879,41 @@ def time_graph(args, fn, dist, local, device, steps):
     return ms, clocks.summary()
 
 
-def prefill_object(args, pre, ms, step_ms, steps, world, clocks, with_cpu):
-    """Bench sub-object of one prefill workload (kernel time = step time: one
-    launch per step)."""
+def prefill_parts(args, pre, dist, device):
+    """(sconv ms, paged-kernel ms) of a two-pass prefill call, its two kernels
+    timed apart as the two public calls that launch them on the same layout
+    (PrefillStep.add_parts); None on the fused path."""
+    if not pre.two_pass:
+        return None
+    pre.add_parts(device)
+    parts = time_loop_only(args, [pre.run_part_sconv, pre.run_part_attn], dist, device)
+    del pre.p_kc, pre.p_vc
+    return parts
+
+
+def prefill_roofline(pre, call_ms, parts, clocks):
+    """Roofline of the call's dominant kernel (the paged prefill kernel on the
+    two-pass path, the fused kernel otherwise) and the path record."""
+    kern_ms = parts[1] if parts else call_ms
+    roof = tensor_roofline(pre.flops / (kern_ms * 1e-3) / 1e12, pre.kernel,
+                           MEASURED_TRAFFIC.get(pre.spec.name), clocks)
+    path = {"path": pre.path, "call_ms": call_ms}
+    if parts:
+        path.update({"sconv_ms": parts[0], "attn_prefill_paged_ms": parts[1],
+                     "kernel_timing": "the call's two kernels timed apart, as the public "
+                                      "sconv append and paged prefill on the same block layout"})
+    return roof, path
+
+
+def prefill_object(args, pre, ms, step_ms, steps, world, clocks, with_cpu, dist=None,
+                   device=None):
+    """Bench sub-object of one prefill workload on the automatic path."""
     tflops = pre.flops / (ms * 1e-3) / 1e12
+    parts = prefill_parts(args, pre, dist, device)
+    roof, path = prefill_roofline(pre, ms, parts, clocks)
     obj = {"workload": pre.spec.name, "value": tflops * world, "unit": "TFLOP/s",
-           "ms_per_step": step_ms, "steps": steps, "gpu_launches": steps,
-           "flops_per_step": pre.flops,
-           "roofline": tensor_roofline(tflops, "attn_prefill_pair_kernel",
-                                       MEASURED_TRAFFIC.get(pre.spec.name), clocks),
+           "ms_per_step": step_ms, "steps": steps, "gpu_launches": steps * pre.launches,
+           "flops_per_step": pre.flops, "prefill_path": path, "roofline": roof,
            "clocks": clocks}
     if with_cpu:
         v, desc, thr = oracle_prefill_sample(pre.spec, args.cpu_seconds)
@@ -916,8 +997,8 @@ def main():
         i = 1
         tflops = pre.flops / (pre_ms * 1e-3) / 1e12 * world
         line.update({"value": tflops, "unit": "TFLOP/s"})
-        line["roofline"] = tensor_roofline(tflops / world, "attn_prefill_pair_kernel",
-                                           MEASURED_TRAFFIC.get(pre.spec.name), clocks)
+        line["roofline"], line["prefill_path"] = prefill_roofline(
+            pre, pre_ms, prefill_parts(args, pre, dist, device), clocks)
     if dec:
         app_ms, attn_ms = per_fn[i], per_fn[i + 1]
         dec_obj = decode_object(dec, app_ms, attn_ms, app_ms + attn_ms, args.steps, world,
@@ -955,15 +1036,27 @@ def main():
     line["clocks"] = clocks
 
     if not args.workload:
-        # the same fused prefill also writing the paged cache and the sconv
-        # state in the same pass, timed on its own after the step
+        # the same prefill on the fused kernel (sconv applied to each key/value
+        # tile on its way to the tensor cores), timed on its own after the step
+        fu_ms = time_loop_only(args, [pre.run_fused], dist, device)[0]
+        fu = pre.flops / (fu_ms * 1e-3) / 1e12
+        line["prefill_fused"] = {
+            "workload": pre.spec.name, "value": fu * world, "unit": "TFLOP/s",
+            "ms_per_step": fu_ms, "gpu_launches": args.steps,
+            "roofline": tensor_roofline(fu, "attn_prefill_pair_kernel",
+                                        MEASURED_TRAFFIC.get(pre.spec.name + " fused"), clocks)}
+        # the same prefill also writing the paged cache and the sconv state,
+        # on the automatic path and on the fused kernel
         pre.add_cache(device)
-        f_ms = time_loop_only(args, [pre.run_fill], dist, device)[0]
+        f_ms, ff_ms = time_loop_only(args, [pre.run_fill, pre.run_fill_fused], dist, device)
         line["prefill_fills_cache"] = {
             "workload": pre.spec.name, "value": pre.flops / (f_ms * 1e-3) / 1e12 * world,
-            "unit": "TFLOP/s", "ms_per_step": f_ms, "gpu_launches": args.steps,
+            "unit": "TFLOP/s", "ms_per_step": f_ms, "path": pre.path,
+            "gpu_launches": args.steps * (pre.launches + 1),
             "cache_bytes_written": pre.spec.B * pre.spec.T * pre.spec.Hkv * 128 * 2 * 2,
-            "plain_ms_per_step": per_fn[0]}
+            "plain_ms_per_step": per_fn[0],
+            "fused": {"value": pre.flops / (ff_ms * 1e-3) / 1e12 * world, "unit": "TFLOP/s",
+                      "ms_per_step": ff_ms, "plain_ms_per_step": fu_ms}}
         # the same prefill shape through the paged cache (sconv append of all
         # keys/values, then the paged prefill), timed on its own after the step
         via = ChunkStep(WORKLOADS[DEFAULT_VIA_CACHE], device)
@@ -1002,7 +1095,8 @@ def main():
                                 "unit": "TFLOP/s", "ms_per_step": pstep}
                 line[name] = obj
             else:
-                line[name] = prefill_object(args, p2, pf[0], pstep, steps, world, pclk, with_cpu)
+                line[name] = prefill_object(args, p2, pf[0], pstep, steps, world, pclk, with_cpu,
+                                            dist, device)
             del p2
             torch.cuda.empty_cache()
         for name in EXTRA_DECODE:
@@ -1020,7 +1114,8 @@ def main():
             line[name] = obj
             del d2
             torch.cuda.empty_cache()
-        line["gpu_launches_all"] = (line["gpu_launches"] + line["prefill_fills_cache"]["gpu_launches"]
+        line["gpu_launches_all"] = (line["gpu_launches"] + line["prefill_fused"]["gpu_launches"]
+                                    + line["prefill_fills_cache"]["gpu_launches"]
                                     + line["prefill_via_cache"]["gpu_launches"]
                                     + sum(line[n]["gpu_launches"] for n in EXTRA_PREFILL + EXTRA_DECODE))
 

@@ -44,6 +44,11 @@
  *    entry outside [0, num_blocks) is reported only through `status`: a
  *    kernel reads block 0 in its place (the rows are finite but wrong) and
  *    skips a write to it.
+ *  - Paged caches: the attention kernels read whole 128-token blocks and give
+ *    the slots past a sequence's length zero weight (0 * x).  Those slots
+ *    must therefore hold finite values (a pool cleared once, or values these
+ *    calls wrote before); NaN or Inf bits there would reach the output.  The
+ *    scratch blocks of the two-pass prefill are zeroed past each end.
  */
 #ifndef INKLING_H
 #define INKLING_H
@@ -126,10 +131,10 @@ typedef struct {
 inkling_status inkling_sconv_kv(const inkling_sconv_params *p, inkling_stream_t stream);
 
 /* --------------------------------------------------------------------------
- * inkling_attn_prefill — prefill attention with the sconv fused into the
- * key/value tile load (Overview, "Attention" and "Short convolution"; the
- * relative term is the FA4 "sheared-bias" kernel named in section
- * Performance).
+ * inkling_attn_prefill — prefill attention over a whole prompt, the sconv of
+ * its keys and values included (Overview, "Attention" and "Short
+ * convolution"; the relative term is the FA4 "sheared-bias" kernel named in
+ * section Performance).
  *
  * Every query row i of every sequence attends to keys j of the same sequence
  * with 0 <= i-j (< window when window > 0).  Keys and values are the sconv of
@@ -149,7 +154,37 @@ inkling_status inkling_sconv_kv(const inkling_sconv_params *p, inkling_stream_t 
  * negative), oldest first, so that inkling_sconv_kv continues the sequence.
  * A block id outside [0, num_blocks) sets INKLING_STATUS_BAD_BLOCK in *status
  * and that tile is not written.  With B = 0 or T = 0 nothing is written.
+ *
+ * Execution path (`path`; results agree within the kernels' rounding, not bit
+ * for bit, since the two paths order the tensor-core sums differently):
+ *  - INKLING_PREFILL_FUSED: one kernel; the sconv is applied to each raw
+ *    key/value tile in shared memory on its way to the tensor cores (and
+ *    written to the cache from there when one is given).  Every thread block
+ *    whose window covers a key tile converts it again.
+ *  - INKLING_PREFILL_TWO_PASS: two kernels.  First the sconv of every key and
+ *    value, written once in the paged layout [block, Hkv, 128, d]: into the
+ *    caller's cache through block_table when one is given (the call is then
+ *    inkling_sconv_kv appending T tokens to empty sequences, with the state
+ *    written as above), else into `workspace`, where sequence b owns blocks
+ *    b*ceil(T/128) ...  Then the paged prefill kernel of
+ *    inkling_attn_prefill_paged over those blocks, every sequence one chunk
+ *    of T rows.  With a cache, a bad block id also spoils the attention rows
+ *    that read that block (block 0 is read in its place).  Needs
+ *    num_blocks*Hkv*128 < 2^31 and B*T*Hq < 2^31 (the workspace blocks
+ *    count when there is no cache); without a cache, workspace_bytes must be
+ *    at least inkling_attn_prefill_workspace_bytes(p).
+ *  - INKLING_PREFILL_AUTO: the two-pass path when T >= INKLING_PREFILL_TWO_PASS_MIN_T
+ *    and it is possible (a cache, or a large enough workspace, and the size
+ *    limits above), else the fused one.  On B200 the two-pass path is 9-12%
+ *    faster from 2048 tokens up (the conversion is done once per token rather
+ *    than once per covering block, for ~1.6% extra HBM traffic), and the
+ *    fused one is faster below ~1024 tokens (one launch instead of two).
  * -------------------------------------------------------------------------- */
+#define INKLING_PREFILL_AUTO 0
+#define INKLING_PREFILL_FUSED 1
+#define INKLING_PREFILL_TWO_PASS 2
+#define INKLING_PREFILL_TWO_PASS_MIN_T 2048
+
 typedef struct {
     const void *q;        /* device [B, T, Hq, d] bf16 */
     const void *k_raw;    /* device [B, T, Hkv, d] bf16, before sconv */
@@ -175,9 +210,21 @@ typedef struct {
     int32_t num_blocks;         /* blocks in the cache pool */
     void *k_state;              /* device [B, 3, Hkv*d] bf16 out, or NULL (with v_state) */
     void *v_state;              /* device [B, 3, Hkv*d] bf16 out, or NULL (with k_state) */
+    /* execution path and scratch */
+    int32_t path;               /* INKLING_PREFILL_AUTO / _FUSED / _TWO_PASS */
+    void *workspace;            /* device scratch of the two-pass path without a cache, or NULL */
+    size_t workspace_bytes;     /* bytes at workspace */
 } inkling_prefill_params;
 
 inkling_status inkling_attn_prefill(const inkling_prefill_params *p, inkling_stream_t stream);
+
+/* Bytes of workspace inkling_attn_prefill(p) uses: 2 * B * ceil(T/128) * Hkv
+ * * 128 * 128 * 2 (post-sconv keys and values in the paged layout) when p's
+ * path is TWO_PASS, or AUTO and T >= INKLING_PREFILL_TWO_PASS_MIN_T, with no
+ * cache given; 0 when the call needs none (the fused path, a cache given, B
+ * or T zero) or p is NULL.  Only the sizes, path and cache pointer of p are
+ * read. */
+size_t inkling_attn_prefill_workspace_bytes(const inkling_prefill_params *p);
 
 /* --------------------------------------------------------------------------
  * inkling_sconv_out — the window-4 short convolution on the attention output

@@ -15,11 +15,12 @@ from .binding import (  # noqa: F401
     decode_num_splits,
     decode_workspace_bytes,
     load_library,
+    prefill_workspace_bytes,
     sconv_kv,
     sconv_out,
     sconv_out_sharded,
 )
 
 __all__ = ["attn_prefill", "attn_prefill_paged", "attn_decode", "attn_decode_static", "sconv_kv", "decode_num_splits",
-           "decode_workspace_bytes", "load_library", "InklingError", "sconv_out",
-           "sconv_out_sharded"]
+           "decode_workspace_bytes", "prefill_workspace_bytes", "load_library", "InklingError",
+           "sconv_out", "sconv_out_sharded"]

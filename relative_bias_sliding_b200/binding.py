@@ -21,6 +21,7 @@ INKLING_OK, INKLING_ERR_INVALID, INKLING_ERR_UNSUPPORTED, INKLING_ERR_CUDA = 0, 
 STATUS_TIMEOUT, STATUS_BAD_BLOCK, STATUS_BAD_LENGTH = 1, 2, 4
 HEAD_DIM = 128
 BLOCK_SIZE = 128
+INKLING_PREFILL_TWO_PASS_MIN_T = 2048
 
 EXPORTED = (
     "inkling_last_error",
@@ -31,6 +32,7 @@ EXPORTED = (
     "inkling_sconv_out_sharded",
     "inkling_attn_prefill",
     "inkling_attn_prefill_paged",
+    "inkling_attn_prefill_workspace_bytes",
     "inkling_attn_decode_workspace_bytes",
     "inkling_attn_decode_num_splits",
     "inkling_attn_decode",
@@ -53,7 +55,12 @@ class PrefillParams(ctypes.Structure):
                 ("out", _P), ("lse", _P), ("status", _P), ("batch", _I), ("seq_len", _I),
                 ("num_q_heads", _I), ("num_kv_heads", _I), ("head_dim", _I), ("window", _I),
                 ("d_max", _I), ("k_cache", _P), ("v_cache", _P), ("block_table", _P),
-                ("max_blocks", _I), ("num_blocks", _I), ("k_state", _P), ("v_state", _P)]
+                ("max_blocks", _I), ("num_blocks", _I), ("k_state", _P), ("v_state", _P),
+                ("path", _I), ("workspace", _P), ("workspace_bytes", ctypes.c_size_t)]
+
+
+# inkling_attn_prefill execution paths (INKLING_PREFILL_*)
+PREFILL_PATHS = {"auto": 0, "fused": 1, "two_pass": 2}
 
 
 class SconvOutParams(ctypes.Structure):
@@ -113,6 +120,8 @@ def load_library(path: str = LIB_PATH):
         lib.inkling_sconv_kv.restype = ctypes.c_int
         lib.inkling_attn_prefill.argtypes = [ctypes.POINTER(PrefillParams), _P]
         lib.inkling_attn_prefill.restype = ctypes.c_int
+        lib.inkling_attn_prefill_workspace_bytes.argtypes = [ctypes.POINTER(PrefillParams)]
+        lib.inkling_attn_prefill_workspace_bytes.restype = ctypes.c_size_t
         lib.inkling_sconv_out.argtypes = [ctypes.POINTER(SconvOutParams), _P]
         lib.inkling_sconv_out.restype = ctypes.c_int
         lib.inkling_sconv_out_sharded.argtypes = [ctypes.POINTER(SconvOutShardedParams), _P]
@@ -190,13 +199,21 @@ def sconv_kv(k_new, v_new, w_k, w_v, k_state, v_state, k_cache, v_cache, block_t
 
 def attn_prefill(q, k_raw, v_raw, w_k, w_v, bias, window=0, out=None, lse=None, status=None,
                  stream=None, k_cache=None, v_cache=None, block_table=None, k_state=None,
-                 v_state=None):
-    """Prefill attention with fused sconv; returns ``out`` [B, T, Hq, d] bf16.
+                 v_state=None, path="auto", workspace=None):
+    """Prefill attention over whole prompts, the sconv of the raw keys/values
+    included; returns ``out`` [B, T, Hq, d] bf16.
 
     With ``k_cache``, ``v_cache`` [num_blocks, Hkv, 128, d] and ``block_table``
-    [B, max_blocks] the same pass writes the post-sconv keys/values of tokens
+    [B, max_blocks] the call also writes the post-sconv keys/values of tokens
     0..T-1 into the paged cache; with ``k_state``, ``v_state`` [B, 3, Hkv*d]
-    it writes the new sconv state."""
+    it writes the new sconv state.
+
+    ``path``: "fused" (one kernel, the sconv applied to each tile on its way
+    to the tensor cores), "two_pass" (the sconv written once in the paged
+    layout, then the paged prefill kernel) or "auto" (the library's choice by
+    length).  Without a cache the two-pass path needs scratch: ``workspace``
+    (a uint8 CUDA tensor of at least ``prefill_workspace_bytes`` bytes), or
+    one is allocated here."""
     bf, f32 = torch.bfloat16, torch.float32
     _dev(q, bf, "q", 4), _dev(k_raw, bf, "k_raw", 4), _dev(v_raw, bf, "v_raw", 4)
     B, T, Hq, d = q.shape
@@ -238,12 +255,34 @@ def attn_prefill(q, k_raw, v_raw, w_k, w_v, bias, window=0, out=None, lse=None, 
             _dev(t, bf, n, 3)
             if t.shape != (B, 3, Hkv * d):
                 raise ValueError(f"{n} must be [{B}, 3, {Hkv * d}]")
+    if path not in PREFILL_PATHS:
+        raise ValueError(f"path must be one of {sorted(PREFILL_PATHS)}")
     p = PrefillParams(_ptr(q), _ptr(k_raw), _ptr(v_raw), _ptr(w_k), _ptr(w_v), _ptr(bias),
                       _ptr(out), _ptr(lse), _ptr(status), B, T, Hq, Hkv, d, int(window), d_max,
                       _ptr(k_cache), _ptr(v_cache), _ptr(block_table), max_blocks, num_blocks,
-                      _ptr(k_state), _ptr(v_state))
-    _check(load_library().inkling_attn_prefill(ctypes.byref(p), _stream(stream)))
+                      _ptr(k_state), _ptr(v_state), PREFILL_PATHS[path], None, 0)
+    lib = load_library()
+    need = lib.inkling_attn_prefill_workspace_bytes(ctypes.byref(p))
+    if need:
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        _dev(workspace, torch.uint8, "workspace", 1)
+        p.workspace, p.workspace_bytes = _ptr(workspace), workspace.numel()
+    _check(lib.inkling_attn_prefill(ctypes.byref(p), _stream(stream)))
     return out
+
+
+def prefill_workspace_bytes(batch, seq_len, num_q_heads, num_kv_heads, path="auto",
+                            with_cache=False):
+    """Bytes of scratch ``attn_prefill`` uses for these sizes and path (0 when
+    it needs none: the fused path, or a cache given)."""
+    if path not in PREFILL_PATHS:
+        raise ValueError(f"path must be one of {sorted(PREFILL_PATHS)}")
+    p = PrefillParams()
+    p.batch, p.seq_len, p.num_q_heads, p.num_kv_heads = batch, seq_len, num_q_heads, num_kv_heads
+    p.head_dim, p.path = 128, PREFILL_PATHS[path]
+    p.k_cache = 16 if with_cache else None  # only tested against NULL
+    return int(load_library().inkling_attn_prefill_workspace_bytes(ctypes.byref(p)))
 
 
 def sconv_out(x, w, state=None, out=None, stream=None):

@@ -9,7 +9,8 @@
 #include "common.cuh"
 
 namespace inkling {
-cudaError_t launch_sconv_kv(const inkling_sconv_params &p, cudaStream_t stream);
+cudaError_t launch_sconv_kv(const inkling_sconv_params &p, cudaStream_t stream,
+                            bool zero_hist = false);
 cudaError_t launch_attn_prefill(const inkling_prefill_params &p, const CUtensorMap *maps,
                                 cudaStream_t stream);
 cudaError_t launch_sconv_out(const inkling_sconv_out_params &p, cudaStream_t stream);
@@ -21,7 +22,7 @@ cudaError_t launch_attn_decode_mq(const inkling_decode_params &p, int splits, in
                                   cudaStream_t stream);
 cudaError_t launch_attn_prefill_paged(const inkling_prefill_paged_params &p, const CUtensorMap &tm_q,
                                       const CUtensorMap &tm_k, const CUtensorMap &tm_v,
-                                      cudaStream_t stream);
+                                      cudaStream_t stream, int dense_T = 0);
 cudaError_t launch_attn_prefill_pair(const inkling_prefill_params &p, const CUtensorMap *maps,
                                      cudaStream_t stream);
 cudaError_t launch_attn_decode(const inkling_decode_params &p, int splits, int s_whole,
@@ -241,6 +242,113 @@ inkling_status validate_decode(const inkling_decode_params *p) {
     return INKLING_OK;
 }
 
+// Tensor maps of the paged prefill kernel: q [rows, Hq, 128] seen as (d,
+// head, row), one box = 128 rows x 64 d of one head; the caches as (d, rows),
+// one box = one 128-token (block, kv head) x 64 d.
+inkling_status paged_maps(const void *q, long rows, int Hq, const void *k_cache,
+                          const void *v_cache, long num_blocks, int Hkv, CUtensorMap *tm_q,
+                          CUtensorMap *tm_k, CUtensorMap *tm_v) {
+    inkling_status st;
+    {
+        cuuint64_t dims[3] = {128, (cuuint64_t)Hq, (cuuint64_t)rows};
+        cuuint64_t str[2] = {256, (cuuint64_t)Hq * 256};
+        cuuint32_t box[3] = {64, 1, 128};
+        if ((st = make_map(tm_q, q, 3, dims, str, box)) != INKLING_OK) return st;
+    }
+    const cuuint64_t crows = (cuuint64_t)num_blocks * Hkv * 128;
+    cuuint64_t dims[2] = {128, crows};
+    cuuint64_t str[1] = {256};
+    cuuint32_t box[2] = {64, 128};
+    if ((st = make_map(tm_k, k_cache, 2, dims, str, box)) != INKLING_OK) return st;
+    return make_map(tm_v, v_cache, 2, dims, str, box);
+}
+
+// The two-pass dense prefill: blocks per sequence of the scratch cache, its
+// bytes, and whether the sizes fit the paged kernel's and the append's limits.
+long scratch_blocks_per_seq(const inkling_prefill_params *p) { return (p->seq_len + 127) / 128; }
+
+size_t scratch_bytes(const inkling_prefill_params *p) {
+    return 2ull * (size_t)p->batch * (size_t)scratch_blocks_per_seq(p) * (size_t)p->num_kv_heads *
+           128 * 128 * 2;
+}
+
+bool two_pass_fits(const inkling_prefill_params *p) {
+    const long pool = p->k_cache ? (long)p->num_blocks : (long)p->batch * scratch_blocks_per_seq(p);
+    return p->seq_len <= (1 << 20) && pool * p->num_kv_heads * 128 < (1L << 31) &&
+           (long)p->batch * p->seq_len * p->num_q_heads < (1L << 31) &&
+           (long)p->batch * scratch_blocks_per_seq(p) <= 0x7fffffffL;
+}
+
+bool wants_two_pass(const inkling_prefill_params *p) {
+    return p->path == INKLING_PREFILL_TWO_PASS ||
+           (p->path == INKLING_PREFILL_AUTO && p->seq_len >= INKLING_PREFILL_TWO_PASS_MIN_T);
+}
+
+// Pass 1: the sconv of all T raw keys/values of every sequence, zero history,
+// into the paged layout (the caller's cache through its block table, else the
+// scratch with sequence b on blocks b*nb ...), the state written when given.
+// Pass 2: the paged prefill kernel with every sequence one chunk of T rows.
+inkling_status prefill_two_pass(const inkling_prefill_params *p, cudaStream_t stream) {
+    const bool cache = p->k_cache != nullptr;
+    const int nb = (int)scratch_blocks_per_seq(p);
+    void *kc = cache ? p->k_cache : p->workspace;
+    void *vc = cache ? p->v_cache : (void *)((char *)p->workspace + scratch_bytes(p) / 2);
+    const int32_t *table = cache ? p->block_table : nullptr;
+    const int max_blocks = cache ? p->max_blocks : nb;
+    const int num_blocks = cache ? p->num_blocks : p->batch * nb;
+
+    inkling_sconv_params sp = {};
+    sp.k_new = p->k_raw;
+    sp.v_new = p->v_raw;
+    sp.w_k = p->w_k;
+    sp.w_v = p->w_v;
+    sp.k_state = p->k_state;
+    sp.v_state = p->v_state;
+    sp.k_cache = kc;
+    sp.v_cache = vc;
+    sp.block_table = table;
+    sp.seq_lens = nullptr;
+    sp.status = p->status;
+    sp.num_seqs = p->batch;
+    sp.n_new = p->seq_len;
+    sp.num_kv_heads = p->num_kv_heads;
+    sp.head_dim = INKLING_HEAD_DIM;
+    sp.max_blocks = max_blocks;
+    sp.num_blocks = num_blocks;
+
+    inkling_prefill_paged_params pp = {};
+    pp.q = p->q;
+    pp.cu_q = nullptr;
+    pp.k_cache = kc;
+    pp.v_cache = vc;
+    pp.block_table = table;
+    pp.seq_lens = nullptr;
+    pp.bias = p->bias;
+    pp.out = p->out;
+    pp.lse = p->lse;
+    pp.status = p->status;
+    pp.num_seqs = p->batch;
+    pp.total_q = p->batch * p->seq_len;
+    pp.max_q = p->seq_len;
+    pp.num_q_heads = p->num_q_heads;
+    pp.num_kv_heads = p->num_kv_heads;
+    pp.head_dim = INKLING_HEAD_DIM;
+    pp.max_blocks = max_blocks;
+    pp.num_blocks = num_blocks;
+    pp.window = p->window;
+    pp.d_max = p->d_max;
+
+    CUtensorMap tm_q, tm_k, tm_v;
+    inkling_status st = paged_maps(p->q, (long)p->batch * p->seq_len, p->num_q_heads, kc, vc,
+                                   num_blocks, p->num_kv_heads, &tm_q, &tm_k, &tm_v);
+    if (st != INKLING_OK) return st;
+    cudaError_t e = launch_sconv_kv(sp, stream, /*zero_hist=*/true);
+    if (e != cudaSuccess) return cuda_fail(e, "attn_prefill (two-pass) sconv launch");
+    e = launch_attn_prefill_paged(pp, tm_q, tm_k, tm_v, stream, p->seq_len);
+    if (e != cudaSuccess) return cuda_fail(e, "attn_prefill (two-pass) paged launch");
+    return INKLING_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -327,8 +435,27 @@ inkling_status inkling_attn_prefill(const inkling_prefill_params *p, inkling_str
         return fail(INKLING_ERR_INVALID, "k_state and v_state go together");
     if (p->k_state && (!aligned16(p->k_state) || !aligned16(p->v_state)))
         return fail(INKLING_ERR_INVALID, "states must be 16-byte aligned");
+    if (p->path < INKLING_PREFILL_AUTO || p->path > INKLING_PREFILL_TWO_PASS)
+        return fail(INKLING_ERR_INVALID, "path must be INKLING_PREFILL_AUTO, _FUSED or _TWO_PASS");
+    if (p->workspace && !aligned16(p->workspace))
+        return fail(INKLING_ERR_INVALID, "workspace must be 16-byte aligned");
+    bool two_pass = false;
+    if (wants_two_pass(p)) {
+        const bool room = p->k_cache || (p->workspace && p->workspace_bytes >= scratch_bytes(p));
+        if (p->path == INKLING_PREFILL_TWO_PASS) {
+            if (!two_pass_fits(p))
+                return fail(INKLING_ERR_UNSUPPORTED,
+                            "two-pass prefill: T above 2^20, or cache rows / B*T*Hq above 2^31");
+            if (!room)
+                return fail(INKLING_ERR_INVALID,
+                            "two-pass prefill without a cache needs a workspace of %zu bytes",
+                            scratch_bytes(p));
+        }
+        two_pass = room && two_pass_fits(p);
+    }
     inkling_status st = check_device(nullptr);
     if (st != INKLING_OK) return st;
+    if (two_pass) return prefill_two_pass(p, (cudaStream_t)stream);
 
     const cuuint64_t T = (cuuint64_t)p->seq_len, B = (cuuint64_t)p->batch;
     const cuuint64_t Hq = (cuuint64_t)p->num_q_heads, Hkv = (cuuint64_t)p->num_kv_heads;
@@ -458,26 +585,20 @@ inkling_status inkling_attn_prefill_paged(const inkling_prefill_paged_params *p,
     inkling_status st = check_device(nullptr);
     if (st != INKLING_OK) return st;
     CUtensorMap tm_q, tm_k, tm_v;
-    {
-        // q [total_q, Hq, 128] seen as (d, head, row): one box = 128 rows x 64 d of one head
-        const cuuint64_t Hq = (cuuint64_t)p->num_q_heads;
-        cuuint64_t dims[3] = {128, Hq, (cuuint64_t)p->total_q};
-        cuuint64_t str[2] = {256, Hq * 256};
-        cuuint32_t box[3] = {64, 1, 128};
-        if ((st = make_map(&tm_q, p->q, 3, dims, str, box)) != INKLING_OK) return st;
-    }
-    {
-        // caches as (d, rows): one box = one 128-token (block, kv head) x 64 d
-        const cuuint64_t rows = (cuuint64_t)p->num_blocks * p->num_kv_heads * 128;
-        cuuint64_t dims[2] = {128, rows};
-        cuuint64_t str[1] = {256};
-        cuuint32_t box[2] = {64, 128};
-        if ((st = make_map(&tm_k, p->k_cache, 2, dims, str, box)) != INKLING_OK) return st;
-        if ((st = make_map(&tm_v, p->v_cache, 2, dims, str, box)) != INKLING_OK) return st;
-    }
+    if ((st = paged_maps(p->q, p->total_q, p->num_q_heads, p->k_cache, p->v_cache, p->num_blocks,
+                         p->num_kv_heads, &tm_q, &tm_k, &tm_v)) != INKLING_OK)
+        return st;
     cudaError_t e = launch_attn_prefill_paged(*p, tm_q, tm_k, tm_v, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "attn_prefill_paged launch");
     return INKLING_OK;
+}
+
+size_t inkling_attn_prefill_workspace_bytes(const inkling_prefill_params *p) {
+    if (!p || p->batch <= 0 || p->seq_len <= 0 || p->num_kv_heads < 1 || p->num_q_heads < 1 ||
+        p->k_cache || !wants_two_pass(p))
+        return 0;
+    if (p->path == INKLING_PREFILL_AUTO && !two_pass_fits(p)) return 0;
+    return scratch_bytes(p);
 }
 
 size_t inkling_attn_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_splits) {

@@ -20,6 +20,13 @@
 // block table), 13 TMEM allocator and MMA issuer, 8-11 and 14-15 idle.
 // Key/value stages: 2.  Rows of the last query tile past the chunk end are
 // computed but not stored.
+//
+// The same kernel is the second pass of the two-pass dense prefill
+// (inkling_attn_prefill): there every sequence is one chunk of T rows over an
+// empty history, so cu_q and seq_lens are NULL (sequence s has rows s*T ..
+// s*T+T-1 and length T), the block table is the caller's cache table or NULL
+// for the scratch cache (sequence s owns blocks s*max_blocks ... in order),
+// and the row log-sum-exp goes to the dense [B, Hq, T] layout.
 #include "prefill_common.cuh"
 
 namespace inkling {
@@ -46,10 +53,11 @@ enum {
 
 struct PagedArgs {
     PrefillArgs pa;  // bias, d_max, window, status, Hq, Hkv (the softmax role's view)
-    const int32_t *cu_q, *block_table, *seq_lens;
+    const int32_t *cu_q, *block_table, *seq_lens;  // cu_q / seq_lens NULL: dense rows
     uint16_t *out;
     float *lse;
     int S, max_blocks, num_blocks, nqb;
+    int dense_T;  // rows (and length) of every sequence when cu_q is NULL
 };
 
 // Epilogue of a chunk row: 16-byte global stores of the rows inside the chunk.
@@ -59,6 +67,13 @@ struct RowStoreEpilogue {
     long row0;       // packed row index of tile row 0
     int rows_valid;  // tile rows inside the chunk
     int Hq, h;
+    int dense_T;     // 0: lse [rows, Hq]; else lse [B, Hq, T] with T = dense_T
+    INK_DEV long lse_at(int u) const {
+        const long r = row0 + u;
+        if (!dense_T) return r * Hq + h;
+        const long b = r / dense_T;
+        return (b * Hq + h) * dense_T + (r - b * dense_T);
+    }
     INK_DEV void operator()(bool have_o, int u, int, float l, float m_ref, uint32_t o_col,
                             volatile int *) const {
         const bool store = u < rows_valid;
@@ -69,14 +84,14 @@ struct RowStoreEpilogue {
                 const uint32_t nb = 0x7fc07fc0u;
 #pragma unroll
                 for (int c = 0; c < 16; ++c) *(uint4 *)(dst + c * 8) = make_uint4(nb, nb, nb, nb);
-                if (lse) lse[(row0 + u) * Hq + h] = __int_as_float(0x7fc00000);
+                if (lse) lse[lse_at(u)] = __int_as_float(0x7fc00000);
             }
             return;  // warp-uniform: emit_row's TMEM loads need the whole warp
         }
         emit_row(o_col, l, [&](int c, uint4 v) {
             if (store) *(uint4 *)(dst + c * 8) = v;
         });
-        if (lse && store) lse[(row0 + u) * Hq + h] = (l > 0.f) ? m_ref + __logf(l) : -INFINITY;
+        if (lse && store) lse[lse_at(u)] = (l > 0.f) ? m_ref + __logf(l) : -INFINITY;
     }
 };
 
@@ -97,9 +112,10 @@ attn_prefill_paged_kernel(const __grid_constant__ CUtensorMap tm_q,
     const int kvh = grp % a.Hkv;
     const int qb = g.nqb - 1 - rem / G;
     const int h = kvh * G + rem % G;
-    const int q_begin = g.cu_q[s];
-    const int n = g.cu_q[s + 1] - q_begin;  // new tokens (query rows) of this sequence
-    const int L = g.seq_lens[s];
+    const bool dense = g.cu_q == nullptr;
+    const int q_begin = dense ? s * g.dense_T : g.cu_q[s];
+    const int n = dense ? g.dense_T : g.cu_q[s + 1] - q_begin;  // query rows of this sequence
+    const int L = g.seq_lens ? g.seq_lens[s] : g.dense_T;
     const int base = L - n;                 // position of the first new token
     if (n < 0 || base < 0 || L > g.max_blocks * 128) {
         if (threadIdx.x == 0 && qb == 0 && h == 0) report_status(a.status, INKLING_STATUS_BAD_LENGTH);
@@ -153,7 +169,8 @@ attn_prefill_paged_kernel(const __grid_constant__ CUtensorMap tm_q,
             softmax_role(a, (float *)(smem + PG_BIAS) + t * 2 * kBiasBuf, &bar[G_SFULL],
                          &bar[G_ODONE], abort_flag, tbase, t, h, base + r0[t], L, lo[t], hi[t],
                          3 + t, 0, 0u, [&](int tt) { mbar_arrive(&bar[G_PFULL + tt]); },
-                         RowStoreEpilogue{g.out, g.lse, (long)q_begin + r0[t], n - r0[t], a.Hq, h});
+                         RowStoreEpilogue{g.out, g.lse, (long)q_begin + r0[t], n - r0[t], a.Hq, h,
+                                          dense ? g.dense_T : 0});
     } else if (warp < 12) {
         setmaxnreg_dec80();
     } else {
@@ -172,7 +189,8 @@ attn_prefill_paged_kernel(const __grid_constant__ CUtensorMap tm_q,
             for (int nt = ulo; nt <= uhi; ++nt) {
                 const int it = nt - ulo, st = it & 1;
                 const uint32_t ph = ((it >> 1) & 1) ^ 1;
-                int blk = g.block_table[(long)s * g.max_blocks + nt];
+                int blk = g.block_table ? g.block_table[(long)s * g.max_blocks + nt]
+                                        : s * g.max_blocks + nt;
                 if (blk < 0 || blk >= g.num_blocks) {
                     report_status(a.status, INKLING_STATUS_BAD_BLOCK);
                     blk = 0;  // keep the pipeline running on a valid block
@@ -289,7 +307,7 @@ attn_prefill_paged_kernel(const __grid_constant__ CUtensorMap tm_q,
 
 cudaError_t launch_attn_prefill_paged(const inkling_prefill_paged_params &p, const CUtensorMap &tm_q,
                                       const CUtensorMap &tm_k, const CUtensorMap &tm_v,
-                                      cudaStream_t stream) {
+                                      cudaStream_t stream, int dense_T) {
     PagedArgs g = {};
     g.pa.bias = p.bias;
     g.pa.status = p.status;
@@ -306,6 +324,7 @@ cudaError_t launch_attn_prefill_paged(const inkling_prefill_paged_params &p, con
     g.max_blocks = p.max_blocks;
     g.num_blocks = p.num_blocks;
     g.nqb = (p.max_q + kQRows - 1) / kQRows;
+    g.dense_T = dense_T;
     const long grid = (long)g.S * p.num_q_heads * g.nqb;
     if (grid == 0) return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(attn_prefill_paged_kernel,

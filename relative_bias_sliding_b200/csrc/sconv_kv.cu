@@ -15,6 +15,13 @@ namespace inkling {
 // (old state, new tokens), after it has read the old one; no other thread
 // touches the state.  Memory-bound: 16-byte loads and stores, one pass, 8
 // tokens' loads in flight per thread.
+//
+// The two-pass prefill runs the same kernel on a whole prompt with three
+// internal modes that the public append never takes: zero_hist (zero raw
+// history before the first new token, the old state not read; a NULL state is
+// then not written either), seq_lens NULL (every length is n_new) and
+// block_table NULL (scratch blocks: sequence s owns blocks s*max_blocks ... in
+// order, and the slots past its end in its last block are zeroed).
 constexpr int kRun = 32;
 
 __global__ void __launch_bounds__(128)
@@ -23,7 +30,8 @@ sconv_kv_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new
                 uint4 *__restrict__ k_state, uint4 *__restrict__ v_state,
                 uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache,
                 const int32_t *__restrict__ block_table, const int32_t *__restrict__ seq_lens,
-                int32_t *status, int S, int n_new, int Hkv, int max_blocks, int num_blocks) {
+                int32_t *status, int S, int n_new, int Hkv, int max_blocks, int num_blocks,
+                bool zero_hist) {
     const int chunks = Hkv * 16;  // 8-channel chunks per token (C = Hkv*128)
     const int runs = (n_new + kRun - 1) / kRun;
     const long gid = (long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -38,7 +46,7 @@ sconv_kv_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new
     uint4 *state = which ? v_state : k_state;
     uint4 *cache = which ? v_cache : k_cache;
 
-    const int L = seq_lens[s];
+    const int L = seq_lens ? seq_lens[s] : n_new;
     if (L < n_new || L > max_blocks * 128) {
         report_status(status, INKLING_STATUS_BAD_LENGTH);
         return;
@@ -53,7 +61,9 @@ sconv_kv_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new
     const int t0 = run * kRun, t1 = min(n_new, t0 + kRun);
     auto new_tok = [&](int t) { return xin[((long)s * n_new + t) * chunks + chunk]; };
     uint4 r3, r2, r1;
-    if (run == 0) {
+    if (run == 0 && zero_hist) {
+        r3 = r2 = r1 = make_uint4(0u, 0u, 0u, 0u);
+    } else if (run == 0) {
         r3 = state[((long)s * 3 + 0) * chunks + chunk];
         r2 = state[((long)s * 3 + 1) * chunks + chunk];
         r1 = state[((long)s * 3 + 2) * chunks + chunk];
@@ -73,8 +83,11 @@ sconv_kv_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new
     // most two 128-token blocks, whose ids are read once
     const int pfirst = L - n_new + t0;
     const int q0 = pfirst >> 7, q1 = (L - n_new + t1 - 1) >> 7;
-    const int blk0 = block_table[(long)s * max_blocks + q0];
-    const int blk1 = (q1 != q0) ? block_table[(long)s * max_blocks + q1] : blk0;
+    auto block_of = [&](int q) {
+        return block_table ? block_table[(long)s * max_blocks + q] : s * max_blocks + q;
+    };
+    const int blk0 = block_of(q0);
+    const int blk1 = (q1 != q0) ? block_of(q1) : blk0;
     const bool bad0 = blk0 < 0 || blk0 >= num_blocks, bad1 = blk1 < 0 || blk1 >= num_blocks;
     if (bad0 || bad1) report_status(status, INKLING_STATUS_BAD_BLOCK);
     // 8 tokens' loads in flight, then their convolutions in order
@@ -97,7 +110,15 @@ sconv_kv_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new
             for (int e = 0; e < 8; ++e) { h3[e] = h2[e]; h2[e] = h1[e]; h1[e] = x[e]; }
         }
     }
-    if (run == 0) {
+    if (!block_table && run == runs - 1 && (L & 127)) {
+        // scratch blocks: zero the slots past the sequence end in its last
+        // block (the attention reads whole blocks and multiplies those slots
+        // by zero probabilities, which stale NaN or Inf bits would survive)
+        const long blk = (long)s * max_blocks + ((L - 1) >> 7);
+        uint4 *dst = cache + ((blk * Hkv + kvh) * 128) * 16 + e16;
+        for (int slot = L & 127; slot < 128; ++slot) dst[(long)slot * 16] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (run == 0 && state) {
         // new state: the last 3 of (old state s3 s2 s1, new tokens 0..n_new-1)
         uint4 ns[3];
 #pragma unroll
@@ -110,7 +131,7 @@ sconv_kv_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new
     }
 }
 
-cudaError_t launch_sconv_kv(const inkling_sconv_params &p, cudaStream_t stream) {
+cudaError_t launch_sconv_kv(const inkling_sconv_params &p, cudaStream_t stream, bool zero_hist) {
     const long runs = (p.n_new + kRun - 1) / kRun;
     const long threads = (long)p.num_seqs * 2 * p.num_kv_heads * 16 * runs;
     if (threads == 0) return cudaSuccess;
@@ -120,7 +141,7 @@ cudaError_t launch_sconv_kv(const inkling_sconv_params &p, cudaStream_t stream) 
         (const uint4 *)p.k_new, (const uint4 *)p.v_new, (const float4 *)p.w_k,
         (const float4 *)p.w_v, (uint4 *)p.k_state, (uint4 *)p.v_state, (uint4 *)p.k_cache,
         (uint4 *)p.v_cache, p.block_table, p.seq_lens, p.status, p.num_seqs, p.n_new,
-        p.num_kv_heads, p.max_blocks, p.num_blocks);
+        p.num_kv_heads, p.max_blocks, p.num_blocks, zero_hist);
     return cudaGetLastError();
 }
 

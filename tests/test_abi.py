@@ -50,7 +50,8 @@ int main(void) {{
          sizeof(inkling_prefill_paged_params));
   F(inkling_sconv_params, num_blocks) F(inkling_prefill_params, d_max)
   F(inkling_prefill_params, k_cache) F(inkling_prefill_params, max_blocks)
-  F(inkling_prefill_params, v_state)
+  F(inkling_prefill_params, v_state) F(inkling_prefill_params, path)
+  F(inkling_prefill_params, workspace) F(inkling_prefill_params, workspace_bytes)
   F(inkling_decode_params, num_splits) F(inkling_decode_params, status)
   F(inkling_decode_params, q_len) F(inkling_prefill_paged_params, cu_q)
   F(inkling_prefill_paged_params, max_q) F(inkling_prefill_paged_params, d_max)
@@ -59,6 +60,8 @@ int main(void) {{
   printf("sharded %zu\\n", sizeof(inkling_sconv_out_sharded_params));
   F(inkling_sconv_out_sharded_params, state) F(inkling_sconv_out_sharded_params, n_ranks)
   F(inkling_sconv_out_sharded_params, channels)
+  printf("paths %d%d%d\\n", INKLING_PREFILL_AUTO, INKLING_PREFILL_FUSED, INKLING_PREFILL_TWO_PASS);
+  printf("min_t %d\\n", INKLING_PREFILL_TWO_PASS_MIN_T);
   return 0;
 }}""")
     exe = tmp_path / "sizes"
@@ -70,7 +73,7 @@ int main(void) {{
     assert int(out["decode"]) == ctypes.sizeof(binding.DecodeParams)
     assert int(out["inkling_sconv_params num_blocks"]) == binding.SconvParams.num_blocks.offset
     assert int(out["inkling_prefill_params d_max"]) == binding.PrefillParams.d_max.offset
-    for m in ("k_cache", "max_blocks", "v_state"):
+    for m in ("k_cache", "max_blocks", "v_state", "path", "workspace", "workspace_bytes"):
         assert int(out["inkling_prefill_params " + m]) == getattr(binding.PrefillParams, m).offset
     assert int(out["inkling_decode_params num_splits"]) == binding.DecodeParams.num_splits.offset
     assert int(out["inkling_decode_params status"]) == binding.DecodeParams.status.offset
@@ -84,6 +87,9 @@ int main(void) {{
     assert int(out["sconv_out"]) == ctypes.sizeof(O)
     assert int(out["inkling_sconv_out_params y"]) == O.y.offset
     assert int(out["inkling_sconv_out_params channels"]) == O.channels.offset
+    P = binding.PREFILL_PATHS
+    assert out["paths"] == f"{P['auto']}{P['fused']}{P['two_pass']}"
+    assert int(out["min_t"]) == binding.INKLING_PREFILL_TWO_PASS_MIN_T
     H = binding.SconvOutShardedParams
     assert int(out["sharded"]) == ctypes.sizeof(H)
     for m in ("state", "n_ranks", "channels"):
@@ -117,6 +123,52 @@ def test_workspace_bytes(lib):
     assert f(1, 64, 148) == 64 * 148 * 130 * 4
     assert f(3, 8, 1) == 16
     assert f(-1, 8, 2) == 0 and f(3, 0, 2) == 0 and f(3, 8, 0) == 0 and f(3, 8, 1025) == 0
+
+
+def test_prefill_workspace_bytes(lib):
+    """The two-pass prefill's scratch: post-sconv K and V of ceil(T/128) blocks
+    per sequence; none for the fused path, with a cache, or below the
+    automatic path's length threshold."""
+    f = lib.inkling_attn_prefill_workspace_bytes
+    p = binding.PrefillParams()
+    p.batch, p.seq_len, p.num_q_heads, p.num_kv_heads, p.head_dim = 4, 8192, 64, 8, 128
+    assert f(ctypes.byref(p)) == 2 * 4 * 64 * 8 * 128 * 128 * 2  # auto, 8192 tokens
+    p.path = binding.PREFILL_PATHS["fused"]
+    assert f(ctypes.byref(p)) == 0
+    p.path, p.seq_len = binding.PREFILL_PATHS["auto"], 2047
+    assert f(ctypes.byref(p)) == 0  # below the threshold the automatic path fuses
+    p.seq_len = 2048
+    assert f(ctypes.byref(p)) == 2 * 4 * 16 * 8 * 128 * 128 * 2
+    p.path, p.seq_len, p.batch = binding.PREFILL_PATHS["two_pass"], 300, 3  # ragged: 3 blocks
+    assert f(ctypes.byref(p)) == 2 * 3 * 3 * 8 * 128 * 128 * 2
+    p.k_cache = ctypes.c_void_p(1 << 20)
+    assert f(ctypes.byref(p)) == 0  # the cache is the scratch
+    p.k_cache, p.seq_len = None, 0
+    assert f(ctypes.byref(p)) == 0
+    assert f(None) == 0
+    assert binding.INKLING_PREFILL_TWO_PASS_MIN_T == 2048
+
+
+def test_prefill_path_validation_rejects_before_launch(lib):
+    fake = ctypes.c_void_p(1 << 20)
+    p = binding.PrefillParams()
+    p.batch, p.seq_len, p.num_q_heads, p.num_kv_heads, p.head_dim = 1, 4096, 8, 1, 128
+    for f in ("q", "k_raw", "v_raw", "w_k", "w_v", "bias", "out"):
+        setattr(p, f, fake)
+    p.path = 3
+    assert lib.inkling_attn_prefill(ctypes.byref(p), None) == binding.INKLING_ERR_INVALID
+    assert b"path" in lib.inkling_last_error()
+    p.path = binding.PREFILL_PATHS["two_pass"]
+    assert lib.inkling_attn_prefill(ctypes.byref(p), None) == binding.INKLING_ERR_INVALID
+    assert b"workspace" in lib.inkling_last_error()
+    p.workspace, p.workspace_bytes = fake, 2 * 32 * 128 * 128 * 2 - 16  # one row short
+    assert lib.inkling_attn_prefill(ctypes.byref(p), None) == binding.INKLING_ERR_INVALID
+    assert b"workspace" in lib.inkling_last_error()
+    p.workspace = ctypes.c_void_p((1 << 20) + 8)
+    assert lib.inkling_attn_prefill(ctypes.byref(p), None) == binding.INKLING_ERR_INVALID
+    assert b"16-byte" in lib.inkling_last_error()
+    p.workspace, p.workspace_bytes, p.seq_len = fake, 1 << 40, (1 << 20) + 1
+    assert lib.inkling_attn_prefill(ctypes.byref(p), None) == binding.INKLING_ERR_UNSUPPORTED
 
 
 def test_host_validation_rejects_before_launch(lib):

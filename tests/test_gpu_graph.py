@@ -23,12 +23,16 @@ def _capture(fn):
     return graph
 
 
-@pytest.mark.parametrize("name", ["prefill_tiny_b1_t256", "prefill_swa_b1_t8192"])
-def test_prefill_graph_replay_matches_eager(name):
+@pytest.mark.parametrize("name,T", [("prefill_tiny_b1_t256", 256),
+                                    ("prefill_swa_b1_t8192", 1000),
+                                    ("prefill_swa_b1_t8192", 2500)])
+def test_prefill_graph_replay_matches_eager(name, T):
+    """256 and 1000 tokens take the fused kernel, 2500 the two-pass path (two
+    kernels, with the scratch allocated by the binding during capture)."""
     need_gpu()
     spec = WORKLOADS[name]
-    if name != "prefill_tiny_b1_t256":
-        spec = scaled(spec, T=1000)  # several query blocks and a ragged tail
+    if T != spec.T:
+        spec = scaled(spec, T=T)  # several query blocks and a ragged tail
     t = make_prefill(spec, device="cuda")
     args = (t["q"], t["k_raw"], t["v_raw"], t["w_k"], t["w_v"], t["bias"])
     eager = ink.attn_prefill(*args, window=spec.window)

@@ -1,4 +1,7 @@
-"""tcgen05 prefill (fused sconv) on the GPU against the oracle, plus invariants."""
+"""tcgen05 prefill on the GPU against the oracle, plus invariants, on both
+execution paths: the fused kernel (sconv applied to each key/value tile in
+shared memory) and the two-pass one (sconv written once in the paged layout,
+then the paged prefill kernel)."""
 import numpy as np
 import pytest
 import torch
@@ -8,15 +11,16 @@ import relative_bias_sliding_b200 as ink
 from relative_bias_sliding_b200.inputs import WORKLOADS, make_prefill, scaled
 
 pytestmark = pytest.mark.gpu
+PATHS = ("fused", "two_pass")
 
 
-def _run(t, window, with_lse=True):
+def _run(t, window, with_lse=True, path="auto"):
     dev = {k: v.cuda() for k, v in t.items()}
     B, T, Hq, _ = dev["q"].shape
     lse = torch.empty((B, Hq, T), dtype=torch.float32, device="cuda") if with_lse else None
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = ink.attn_prefill(dev["q"], dev["k_raw"], dev["v_raw"], dev["w_k"], dev["w_v"],
-                           dev["bias"], window=window, lse=lse, status=status)
+                           dev["bias"], window=window, lse=lse, status=status, path=path)
     torch.cuda.synchronize()
     assert status.item() == 0, f"status {status.item()}"
     return out, lse
@@ -33,11 +37,12 @@ def test_prefill_tiny_workload_all_rows(oracle_mod):
     need_gpu()
     spec = WORKLOADS["prefill_tiny_b1_t256"]
     t = make_prefill(spec)
-    out, lse = _run(t, spec.window)
     ref, ref_lse = _oracle_all(oracle_mod, t, spec.window)
-    assert_parity(out, ref, spec.name)
-    got_lse = lse.permute(0, 2, 1).cpu().numpy().reshape(-1)   # [B, T, Hq] order
-    np.testing.assert_allclose(got_lse, ref_lse, rtol=0, atol=2e-3)
+    for path in PATHS:
+        out, lse = _run(t, spec.window, path=path)
+        assert_parity(out, ref, f"{spec.name} {path}")
+        got_lse = lse.permute(0, 2, 1).cpu().numpy().reshape(-1)   # [B, T, Hq] order
+        np.testing.assert_allclose(got_lse, ref_lse, rtol=0, atol=2e-3)
 
 
 @pytest.mark.parametrize("B,T,Hq,Hkv,W,D_max", [
@@ -51,15 +56,19 @@ def test_prefill_tiny_workload_all_rows(oracle_mod):
     (3, 257, 8, 4, 256, 300),    # query block boundary + 1
     (1, 600, 12, 2, 200, 300),   # G = 6: two heads x 256 rows per CTA pair
     (2, 400, 12, 3, 0, 400),     # G = 4, three kv heads: four heads x 128 rows per pair
+    (2, 130, 6, 2, 0, 200),      # G = 3 (single-CTA fused kernel), 2 blocks, 2 rows past one
 ])
 def test_prefill_ragged_and_masks(oracle_mod, B, T, Hq, Hkv, W, D_max):
     need_gpu()
     spec = scaled(WORKLOADS["prefill_tiny_b1_t256"], B=B, T=T, Hq=Hq, Hkv=Hkv, window=W,
                   D_max=D_max, seed=T + W)
     t = make_prefill(spec)
-    out, _ = _run(t, W)
-    ref, _ = _oracle_all(oracle_mod, t, W)
-    assert_parity(out, ref, f"B{B} T{T} Hq{Hq} Hkv{Hkv} W{W} D{D_max}")
+    ref, ref_lse = _oracle_all(oracle_mod, t, W)
+    for path in PATHS:
+        out, lse = _run(t, W, path=path)
+        assert_parity(out, ref, f"B{B} T{T} Hq{Hq} Hkv{Hkv} W{W} D{D_max} {path}")
+        got_lse = lse.permute(0, 2, 1).cpu().numpy().reshape(-1)
+        np.testing.assert_allclose(got_lse, ref_lse, rtol=0, atol=2e-3)
 
 
 @pytest.mark.parametrize("B,T,Hq,Hkv,W", [
@@ -75,30 +84,107 @@ def test_prefill_several_waves_all_rows(oracle_mod, B, T, Hq, Hkv, W):
     spec = scaled(WORKLOADS["prefill_swa_b4_t8192"], B=B, T=T, Hq=Hq, Hkv=Hkv, window=W,
                   D_max=3000, seed=11 + W)
     t = make_prefill(spec)
-    out, lse = _run(t, W)
     ref, ref_lse = _oracle_all(oracle_mod, t, W)
-    assert_parity(out, ref, f"B{B} T{T} Hq{Hq} Hkv{Hkv} W{W}")
-    got_lse = lse.permute(0, 2, 1).cpu().numpy().reshape(-1)
-    np.testing.assert_allclose(got_lse, ref_lse, rtol=0, atol=2e-3)
+    for path in PATHS:
+        out, lse = _run(t, W, path=path)
+        assert_parity(out, ref, f"B{B} T{T} Hq{Hq} Hkv{Hkv} W{W} {path}")
+        got_lse = lse.permute(0, 2, 1).cpu().numpy().reshape(-1)
+        np.testing.assert_allclose(got_lse, ref_lse, rtol=0, atol=2e-3)
 
 
-def test_prefill_window_at_least_T_equals_full():
+@pytest.mark.parametrize("path", PATHS)
+def test_prefill_window_at_least_T_equals_full(path):
     need_gpu()
     spec = scaled(WORKLOADS["prefill_tiny_b1_t256"], T=600, Hq=8, Hkv=2, D_max=700, seed=5)
     t = make_prefill(spec)
-    full, _ = _run(t, 0)
-    win, _ = _run(t, 600)
+    full, _ = _run(t, 0, path=path)
+    win, _ = _run(t, 600, path=path)
     assert torch.equal(full, win)
 
 
-def test_prefill_empty_batch_is_noop():
+@pytest.mark.parametrize("T", [2047, 2048])
+def test_prefill_auto_path_follows_the_length_threshold(T):
+    """The automatic path fuses below 2048 tokens and runs the two passes from
+    there: the library asks for a workspace only from 2048 tokens, and a
+    workspace passed then is written by the first pass.  The two paths give the
+    same bits: the same MMA order and softmax code over the same post-sconv
+    keys and values."""
+    need_gpu()
+    Hq, Hkv = 16, 2
+    spec = scaled(WORKLOADS["prefill_swa_b4_t8192"], B=1, T=T, Hq=Hq, Hkv=Hkv, window=1000,
+                  D_max=3000, seed=T)
+    t = make_prefill(spec)
+    dev = {k: v.cuda() for k, v in t.items()}
+    need = ink.prefill_workspace_bytes(1, T, Hq, Hkv)
+    assert (need > 0) == (T >= 2048)
+    ws = torch.full((max(need, 16),), 0xff, dtype=torch.uint8, device="cuda")
+    lse = torch.empty((1, Hq, T), dtype=torch.float32, device="cuda")
+    auto = ink.attn_prefill(dev["q"], dev["k_raw"], dev["v_raw"], dev["w_k"], dev["w_v"],
+                            dev["bias"], window=1000, lse=lse, workspace=ws)
+    torch.cuda.synchronize()
+    assert bool((ws != 0xff).any()) == (T >= 2048)
+    for path in PATHS:
+        out, lse2 = _run(t, 1000, path=path)
+        assert torch.equal(auto.view(torch.int16), out.view(torch.int16)), path
+        assert torch.equal(lse, lse2), path
+
+
+def test_prefill_two_pass_uses_the_given_workspace(oracle_mod):
+    """With a workspace passed in, the two-pass path writes the post-sconv
+    keys/values there, in the paged layout (sequence b on blocks b*nb ...),
+    bit for bit what the sconv append writes for the same tokens, and zeroes
+    the slots past the end of each sequence's last block: a workspace full of
+    NaN bits gives the oracle's rows."""
+    need_gpu()
+    B, T, Hq, Hkv = 2, 300, 8, 2
+    spec = scaled(WORKLOADS["prefill_tiny_b1_t256"], B=B, T=T, Hq=Hq, Hkv=Hkv, D_max=300, seed=9)
+    t = make_prefill(spec)
+    dev = {k: v.cuda() for k, v in t.items()}
+    nb = (T + 127) // 128
+    need = ink.prefill_workspace_bytes(B, T, Hq, Hkv, path="two_pass")
+    assert need == 2 * B * nb * Hkv * 128 * 128 * 2
+    ws = torch.full((need + 64,), 0xff, dtype=torch.uint8, device="cuda")   # bf16 NaN bits
+    out = ink.attn_prefill(dev["q"], dev["k_raw"], dev["v_raw"], dev["w_k"], dev["w_v"],
+                           dev["bias"], path="two_pass", workspace=ws)
+    kc = torch.zeros((B * nb, Hkv, 128, 128), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    st = torch.zeros((B, 3, Hkv * 128), dtype=torch.bfloat16, device="cuda")
+    st2 = torch.zeros_like(st)
+    bt = torch.arange(B * nb, dtype=torch.int32, device="cuda").reshape(B, nb)
+    ink.sconv_kv(dev["k_raw"], dev["v_raw"], dev["w_k"], dev["w_v"], st, st2, kc, vc, bt,
+                 torch.full((B,), T, dtype=torch.int32, device="cuda"))
+    torch.cuda.synchronize()
+    half = need // 2
+    got_k = ws[:half].view(torch.bfloat16).reshape(kc.shape)
+    got_v = ws[half:need].view(torch.bfloat16).reshape(vc.shape)
+    for b in range(B):
+        for blk in range(nb):
+            n = min(128, T - blk * 128)
+            i = b * nb + blk
+            assert torch.equal(got_k[i, :, :n].view(torch.int16), kc[i, :, :n].view(torch.int16))
+            assert torch.equal(got_v[i, :, :n].view(torch.int16), vc[i, :, :n].view(torch.int16))
+            assert (got_k[i, :, n:].view(torch.int16) == 0).all()
+            assert (got_v[i, :, n:].view(torch.int16) == 0).all()
+    assert (ws[need:] == 0xff).all()   # nothing past the workspace size
+    ref, _, _, _ = oracle_mod.prefill_rows(u16(t["q"]), u16(t["k_raw"]), u16(t["v_raw"]),
+                                           t["w_k"].numpy(), t["w_v"].numpy(), t["bias"].numpy(),
+                                           0, 300)
+    assert_parity(out, ref, "two-pass over a NaN-filled workspace")
+    again = ink.attn_prefill(dev["q"], dev["k_raw"], dev["v_raw"], dev["w_k"], dev["w_v"],
+                             dev["bias"], path="two_pass")   # scratch allocated by the binding
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), again.view(torch.int16))
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_prefill_empty_batch_is_noop(path):
     need_gpu()
     spec = scaled(WORKLOADS["prefill_tiny_b1_t256"], B=1, T=16)
     t = make_prefill(spec)
     dev = {k: v.cuda() for k, v in t.items()}
     out = torch.full((0, 16, 8, 128), 7.0, dtype=torch.bfloat16, device="cuda")
     ink.attn_prefill(dev["q"][:0], dev["k_raw"][:0], dev["v_raw"][:0], dev["w_k"], dev["w_v"],
-                     dev["bias"], out=out)
+                     dev["bias"], out=out, path=path)
     torch.cuda.synchronize()
 
 
@@ -161,20 +247,27 @@ def _sample_rows(spec, rng, per_head):
                                            ("prefill_full_b1_t32768", 256)])
 def test_prefill_full_size_sampled_rows(oracle_mod, name, per_head):
     """The benchmark workloads at full size, in the benchmark's launch
-    configuration; the oracle computes a sample of rows of every (batch, head)."""
+    configuration (the automatic path, two-pass at these lengths) and on the
+    fused kernel; the oracle computes a sample of rows of every (batch, head),
+    with their log-sum-exp."""
     need_gpu()
     spec = WORKLOADS[name]
     t = make_prefill(spec, device="cuda")
-    status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    out = ink.attn_prefill(t["q"], t["k_raw"], t["v_raw"], t["w_k"], t["w_v"], t["bias"],
-                           window=spec.window, status=status)
-    torch.cuda.synchronize()
-    assert status.item() == 0
     rows = _sample_rows(spec, np.random.default_rng(0), per_head)
-    ref, _, _, _ = oracle_mod.prefill_rows(u16(t["q"]), u16(t["k_raw"]), u16(t["v_raw"]),
-                                           t["w_k"].cpu().numpy(), t["w_v"].cpu().numpy(),
-                                           t["bias"].cpu().numpy(), spec.window, spec.D_max,
-                                           rows)
+    ref, ref_lse, _, _ = oracle_mod.prefill_rows(u16(t["q"]), u16(t["k_raw"]), u16(t["v_raw"]),
+                                                 t["w_k"].cpu().numpy(), t["w_v"].cpu().numpy(),
+                                                 t["bias"].cpu().numpy(), spec.window,
+                                                 spec.D_max, rows)
     r = torch.from_numpy(rows).long().cuda()
-    got = out[r[:, 0], r[:, 2], r[:, 1]].float().cpu().numpy()
-    assert_parity(got, ref, name)
+    lse = torch.empty((spec.B, spec.Hq, spec.T), dtype=torch.float32, device="cuda")
+    for path in ("auto", "fused"):
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        out = ink.attn_prefill(t["q"], t["k_raw"], t["v_raw"], t["w_k"], t["w_v"], t["bias"],
+                               window=spec.window, status=status, lse=lse, path=path)
+        torch.cuda.synchronize()
+        assert status.item() == 0
+        got = out[r[:, 0], r[:, 2], r[:, 1]].float().cpu().numpy()
+        assert_parity(got, ref, f"{name} {path}")
+        got_lse = lse[r[:, 0], r[:, 1], r[:, 2]].cpu().numpy()
+        np.testing.assert_allclose(got_lse, ref_lse, rtol=0, atol=2e-3)
+        del out

@@ -1,6 +1,7 @@
-"""The fused prefill filling the paged cache and the sconv state in the same
-pass: bit for bit what the sconv append writes for the same tokens, and a
-decode that continues from it matches the oracle."""
+"""The prefill filling the paged cache and the sconv state in the same call,
+on both execution paths (fused kernel; sconv append then paged prefill): bit
+for bit what the sconv append writes for the same tokens, and a decode that
+continues from it matches the oracle."""
 import numpy as np
 import pytest
 import torch
@@ -35,7 +36,8 @@ def _setup(B, T, Hq, Hkv, W, D, seed, spare=2):
     (1, 128, 8, 2, 0),       # exactly one block
     (3, 4096, 8, 1, 1024),   # several query blocks per sequence, window
 ])
-def test_prefill_cache_equals_append(B, T, Hq, Hkv, W):
+@pytest.mark.parametrize("path", ["fused", "two_pass"])
+def test_prefill_cache_equals_append(B, T, Hq, Hkv, W, path):
     need_gpu()
     spec, t, dev, bt, kc, vc = _setup(B, T, Hq, Hkv, W, 512, seed=T + Hq)
     kc2, vc2 = kc.clone(), vc.clone()
@@ -45,9 +47,9 @@ def test_prefill_cache_equals_append(B, T, Hq, Hkv, W):
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = ink.attn_prefill(dev["q"], dev["k_raw"], dev["v_raw"], dev["w_k"], dev["w_v"],
                            dev["bias"], window=W, status=status, k_cache=kc, v_cache=vc,
-                           block_table=bt, k_state=ks, v_state=vs)
+                           block_table=bt, k_state=ks, v_state=vs, path=path)
     plain = ink.attn_prefill(dev["q"], dev["k_raw"], dev["v_raw"], dev["w_k"], dev["w_v"],
-                             dev["bias"], window=W)
+                             dev["bias"], window=W, path=path)
     # the same tokens appended to empty sequences
     ks2 = torch.zeros((B, 3, C), dtype=torch.bfloat16, device="cuda")
     vs2 = torch.zeros_like(ks2)
@@ -62,7 +64,8 @@ def test_prefill_cache_equals_append(B, T, Hq, Hkv, W):
     assert torch.equal(vs.view(torch.int16), vs2.view(torch.int16))
 
 
-def test_decode_continues_from_prefill_cache(oracle_mod):
+@pytest.mark.parametrize("path", ["fused", "two_pass"])
+def test_decode_continues_from_prefill_cache(oracle_mod, path):
     """Serving order: prefill T tokens (filling cache and state), append one
     token with the sconv append, decode it; the oracle computes row T of the
     T+1-token sequence from the raw keys and values."""
@@ -74,7 +77,8 @@ def test_decode_continues_from_prefill_cache(oracle_mod):
     vs = torch.zeros_like(ks)
     ink.attn_prefill(dev["q"][:, :T].contiguous(), dev["k_raw"][:, :T].contiguous(),
                      dev["v_raw"][:, :T].contiguous(), dev["w_k"], dev["w_v"], dev["bias"],
-                     window=W, k_cache=kc, v_cache=vc, block_table=bt, k_state=ks, v_state=vs)
+                     window=W, k_cache=kc, v_cache=vc, block_table=bt, k_state=ks, v_state=vs,
+                     path=path)
     lens = torch.full((B,), T + 1, dtype=torch.int32, device="cuda")
     ink.sconv_kv(dev["k_raw"][:, T:].contiguous(), dev["v_raw"][:, T:].contiguous(), dev["w_k"],
                  dev["w_v"], ks, vs, kc, vc, bt, lens)
@@ -87,7 +91,12 @@ def test_decode_continues_from_prefill_cache(oracle_mod):
     assert_parity(dec.reshape(B * Hq, 128), ref, "decode after prefill cache fill")
 
 
-def test_prefill_cache_bad_block_is_reported_and_skipped():
+@pytest.mark.parametrize("path", ["fused", "two_pass"])
+def test_prefill_cache_bad_block_is_reported_and_skipped(path):
+    """A block id outside the pool is reported and never written.  The fused
+    kernel attends from its shared-memory tiles, so its rows stay right; the
+    two-pass path reads the keys back from the cache, block 0 in place of the
+    bad one, so only the rows that never see that block are checked."""
     need_gpu()
     B, T, Hq, Hkv = 1, 300, 8, 1
     spec, t, dev, bt, kc, vc = _setup(B, T, Hq, Hkv, 0, 300, seed=5)
@@ -95,12 +104,14 @@ def test_prefill_cache_bad_block_is_reported_and_skipped():
     before = kc.clone()
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = ink.attn_prefill(dev["q"], dev["k_raw"], dev["v_raw"], dev["w_k"], dev["w_v"],
-                           dev["bias"], status=status, k_cache=kc, v_cache=vc, block_table=bt)
+                           dev["bias"], status=status, k_cache=kc, v_cache=vc, block_table=bt,
+                           path=path)
     plain = ink.attn_prefill(dev["q"], dev["k_raw"], dev["v_raw"], dev["w_k"], dev["w_v"],
-                             dev["bias"])
+                             dev["bias"], path=path)
     torch.cuda.synchronize()
     assert status.item() & 2              # INKLING_STATUS_BAD_BLOCK
-    assert torch.equal(out.view(torch.int16), plain.view(torch.int16))
+    rows = slice(None) if path == "fused" else slice(0, 128)   # rows 0..127 see block 0 only
+    assert torch.equal(out[:, rows].view(torch.int16), plain[:, rows].view(torch.int16))
     # the valid blocks were written, the pool is otherwise unchanged
     assert not torch.equal(kc[bt[0, 0]], before[bt[0, 0]])
     untouched = [i for i in range(kc.shape[0]) if i not in (int(bt[0, 0]), int(bt[0, 2]))]
