@@ -53,7 +53,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # 3 warm-up launches; profiles/ holds the summaries and commands).  Remove an
 # entry when its kernel changes until it is captured again.
 MEASURED_TRAFFIC = {
-    "prefill_swa_b4_t8192": 677_133_312 + 499_282_176,   # paged kernel of the two-pass call
+    # the prefill call's dominant kernel: the paged kernel on the two-pass path,
+    # the pair kernel on the fused one (" fused")
+    "prefill_swa_b4_t8192": 677_133_312 + 499_282_176,
     "prefill_swa_b4_t8192 fused": 680_339_712 + 501_876_992,
     "decode_swa_s64": 1_080_809_216 + 3_773_440,
     "decode_mtp9_swa_s64": 1_089_955_584 + 8_819_968,
@@ -200,7 +202,7 @@ class PrefillStep:
     below), plus the fused kernel and the cache-filling variants of the same
     call, and the two passes as separate public calls for their timings."""
 
-    def __init__(self, spec, device):
+    def __init__(self, spec, device, path="auto"):
         import torch
         import relative_bias_sliding_b200 as ink
         from relative_bias_sliding_b200.inputs import make_prefill
@@ -208,7 +210,8 @@ class PrefillStep:
         self.t = make_prefill(spec, device=device)
         self.out = torch.empty_like(self.t["q"])
         self.flops = spec.flops
-        nbytes = ink.prefill_workspace_bytes(spec.B, spec.T, spec.Hq, spec.Hkv)
+        self.path_arg = path
+        nbytes = ink.prefill_workspace_bytes(spec.B, spec.T, spec.Hq, spec.Hkv, path=path)
         self.ws = torch.empty(nbytes, dtype=torch.uint8, device=device) if nbytes else None
         self.two_pass = nbytes > 0
         self.launches = 2 if self.two_pass else 1
@@ -220,7 +223,7 @@ class PrefillStep:
         t = self.t
         ink.attn_prefill(t["q"], t["k_raw"], t["v_raw"], t["w_k"], t["w_v"], t["bias"],
                          window=self.spec.window, out=self.out, stream=stream,
-                         workspace=self.ws)
+                         path=self.path_arg, workspace=self.ws)
 
     def run_fused(self, stream=None):
         import relative_bias_sliding_b200 as ink
@@ -299,6 +302,7 @@ class DecodeStep:
         nbytes = max(16, ink.decode_workspace_bytes(rows, spec.Hq, self.splits))
         self.ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
         self.kv_bytes = kv_bytes_read(spec, t["seq_lens"].cpu())
+        self.cache_bytes = 2 * t["k_cache"].numel() * t["k_cache"].element_size()
         self.launches = 2 + (1 if self.splits > 1 else 0)
 
     def run_append(self, stream=None):
@@ -430,7 +434,7 @@ def e2e_prefill(step, steps, stream):
     def compute(b, s):
         ink.attn_prefill(dev[b]["q"], dev[b]["k_raw"], dev[b]["v_raw"], t["w_k"], t["w_v"],
                          t["bias"], window=step.spec.window, out=outs[b], stream=s,
-                         workspace=step.ws)  # the calls run in order on one stream
+                         path=step.path_arg, workspace=step.ws)  # calls in order on one stream
 
     def d2h(b, s):
         with torch.cuda.stream(s):
@@ -659,6 +663,9 @@ def parse():
     ap.add_argument("--clocks-log-dir", default=None,
                     help="keep the raw nvidia-smi clock samples in this directory")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--prefill-path", default="auto", choices=["auto", "fused", "two_pass"],
+                    help="inkling_attn_prefill path of the timed prefill (default: the library's "
+                         "automatic choice)")
     return ap.parse_args()
 
 
@@ -895,8 +902,9 @@ def prefill_roofline(pre, call_ms, parts, clocks):
     """Roofline of the call's dominant kernel (the paged prefill kernel on the
     two-pass path, the fused kernel otherwise) and the path record."""
     kern_ms = parts[1] if parts else call_ms
+    key = pre.spec.name + ("" if pre.two_pass else " fused")
     roof = tensor_roofline(pre.flops / (kern_ms * 1e-3) / 1e12, pre.kernel,
-                           MEASURED_TRAFFIC.get(pre.spec.name), clocks)
+                           MEASURED_TRAFFIC.get(key), clocks)
     path = {"path": pre.path, "call_ms": call_ms}
     if parts:
         path.update({"sconv_ms": parts[0], "attn_prefill_paged_ms": parts[1],
@@ -964,10 +972,10 @@ def main():
             return run_sconv_out(args, spec, dist, rank, world, local, device)
         if isinstance(spec, ChunkSpec):
             return run_chunk(args, ChunkStep(spec, device), dist, rank, world, local, device)
-        pre = PrefillStep(spec, device) if isinstance(spec, PrefillSpec) else None
+        pre = PrefillStep(spec, device, args.prefill_path) if isinstance(spec, PrefillSpec) else None
         dec = None if pre else DecodeStep(spec, device)
     else:
-        pre = PrefillStep(WORKLOADS[DEFAULT_PREFILL], device)
+        pre = PrefillStep(WORKLOADS[DEFAULT_PREFILL], device, args.prefill_path)
         dec = DecodeStep(WORKLOADS[DEFAULT_DECODE], device)
     fns = []
     if pre:
@@ -1010,10 +1018,17 @@ def main():
             line.update({"value": dec_obj["value"], "unit": "GB/s",
                          "roofline": dec_obj["roofline"]})
             line["decode"] = {k: v for k, v in dec_obj.items() if k != "roofline"}
+    sizes = []
+    if pre:
+        sizes.append(f"prefill q {pre.t['q'].numel() * 2 / 2**20:.0f} MiB")
+    if dec:
+        sizes.append(f"decode K/V cache {dec.cache_bytes / 1e9:.1f} GB")
     line["config"] = {"workload": (pre.spec.name if pre else "") +
                       (" + " if pre and dec else "") + (dec.spec.name if dec else ""),
                       "parallelism": f"replica per GPU x{world}",
-                      "l2": "inputs larger than L2 (prefill q 512 MiB; decode KV 4.4 GB)"}
+                      "l2": "inputs larger than L2 (" + "; ".join(sizes) + ")"}
+    if pre:
+        line["config"]["prefill_path"] = args.prefill_path
     if e2e:
         parts = {p[0]: p[1:] for p in e2e}
         if pre:
@@ -1081,7 +1096,7 @@ def main():
         # the other workloads of the layer, each timed on its own with its
         # roofline and the oracle timed beside it
         for name in EXTRA_PREFILL:
-            p2 = PrefillStep(WORKLOADS[name], device)
+            p2 = PrefillStep(WORKLOADS[name], device, args.prefill_path)
             steps = max(args.steps, 200) if p2.flops < 1e10 else args.steps
             pf, pstep, pclk = time_with_clocks(args, [p2.run], dist, local, device, steps)
             if p2.flops < 1e10:
