@@ -155,8 +155,9 @@ inkling_status inkling_sconv_kv(const inkling_sconv_params *p, inkling_stream_t 
  * A block id outside [0, num_blocks) sets INKLING_STATUS_BAD_BLOCK in *status
  * and that tile is not written.  With B = 0 or T = 0 nothing is written.
  *
- * Execution path (`path`; results agree within the kernels' rounding, not bit
- * for bit, since the two paths order the tensor-core sums differently):
+ * Execution path (`path`).  Both paths give the same bits: the same tensor-core
+ * accumulation order and softmax code over the same post-sconv keys and
+ * values (the sconv arithmetic is shared with inkling_sconv_kv).
  *  - INKLING_PREFILL_FUSED: one kernel; the sconv is applied to each raw
  *    key/value tile in shared memory on its way to the tensor cores (and
  *    written to the cache from there when one is given).  Every thread block

@@ -64,11 +64,16 @@ def test_prefill_ragged_and_masks(oracle_mod, B, T, Hq, Hkv, W, D_max):
                   D_max=D_max, seed=T + W)
     t = make_prefill(spec)
     ref, ref_lse = _oracle_all(oracle_mod, t, W)
+    got = {}
     for path in PATHS:
         out, lse = _run(t, W, path=path)
         assert_parity(out, ref, f"B{B} T{T} Hq{Hq} Hkv{Hkv} W{W} D{D_max} {path}")
         got_lse = lse.permute(0, 2, 1).cpu().numpy().reshape(-1)
         np.testing.assert_allclose(got_lse, ref_lse, rtol=0, atol=2e-3)
+        got[path] = (out, lse)
+    # the two paths give the same bits (same MMA order and softmax code)
+    assert torch.equal(got["fused"][0].view(torch.int16), got["two_pass"][0].view(torch.int16))
+    assert torch.equal(got["fused"][1], got["two_pass"][1])
 
 
 @pytest.mark.parametrize("B,T,Hq,Hkv,W", [
@@ -85,11 +90,15 @@ def test_prefill_several_waves_all_rows(oracle_mod, B, T, Hq, Hkv, W):
                   D_max=3000, seed=11 + W)
     t = make_prefill(spec)
     ref, ref_lse = _oracle_all(oracle_mod, t, W)
+    got = {}
     for path in PATHS:
         out, lse = _run(t, W, path=path)
         assert_parity(out, ref, f"B{B} T{T} Hq{Hq} Hkv{Hkv} W{W} {path}")
         got_lse = lse.permute(0, 2, 1).cpu().numpy().reshape(-1)
         np.testing.assert_allclose(got_lse, ref_lse, rtol=0, atol=2e-3)
+        got[path] = (out, lse)
+    assert torch.equal(got["fused"][0].view(torch.int16), got["two_pass"][0].view(torch.int16))
+    assert torch.equal(got["fused"][1], got["two_pass"][1])
 
 
 @pytest.mark.parametrize("path", PATHS)
@@ -259,8 +268,9 @@ def test_prefill_full_size_sampled_rows(oracle_mod, name, per_head):
                                                  t["bias"].cpu().numpy(), spec.window,
                                                  spec.D_max, rows)
     r = torch.from_numpy(rows).long().cuda()
-    lse = torch.empty((spec.B, spec.Hq, spec.T), dtype=torch.float32, device="cuda")
+    first = None
     for path in ("auto", "fused"):
+        lse = torch.empty((spec.B, spec.Hq, spec.T), dtype=torch.float32, device="cuda")
         status = torch.zeros(1, dtype=torch.int32, device="cuda")
         out = ink.attn_prefill(t["q"], t["k_raw"], t["v_raw"], t["w_k"], t["w_v"], t["bias"],
                                window=spec.window, status=status, lse=lse, path=path)
@@ -270,4 +280,8 @@ def test_prefill_full_size_sampled_rows(oracle_mod, name, per_head):
         assert_parity(got, ref, f"{name} {path}")
         got_lse = lse[r[:, 0], r[:, 1], r[:, 2]].cpu().numpy()
         np.testing.assert_allclose(got_lse, ref_lse, rtol=0, atol=2e-3)
-        del out
+        if first is None:
+            first = (out, lse)
+        else:   # the two paths give the same bits at full size too
+            assert torch.equal(first[0].view(torch.int16), out.view(torch.int16))
+            assert torch.equal(first[1], lse)
