@@ -22,7 +22,7 @@ cudaError_t launch_attn_decode_mq(const inkling_decode_params &p, int splits, in
                                   cudaStream_t stream);
 cudaError_t launch_attn_prefill_paged(const inkling_prefill_paged_params &p, const CUtensorMap &tm_q,
                                       const CUtensorMap &tm_k, const CUtensorMap &tm_v,
-                                      cudaStream_t stream, int dense_T = 0);
+                                      cudaStream_t stream, int dense_T, int sms);
 cudaError_t launch_attn_prefill_pair(const inkling_prefill_params &p, const CUtensorMap *maps,
                                      cudaStream_t stream);
 cudaError_t launch_attn_decode(const inkling_decode_params &p, int splits, int s_whole,
@@ -288,7 +288,7 @@ bool wants_two_pass(const inkling_prefill_params *p) {
 // into the paged layout (the caller's cache through its block table, else the
 // scratch with sequence b on blocks b*nb ...), the state written when given.
 // Pass 2: the paged prefill kernel with every sequence one chunk of T rows.
-inkling_status prefill_two_pass(const inkling_prefill_params *p, cudaStream_t stream) {
+inkling_status prefill_two_pass(const inkling_prefill_params *p, cudaStream_t stream, int sms) {
     const bool cache = p->k_cache != nullptr;
     const int nb = (int)scratch_blocks_per_seq(p);
     void *kc = cache ? p->k_cache : p->workspace;
@@ -344,7 +344,7 @@ inkling_status prefill_two_pass(const inkling_prefill_params *p, cudaStream_t st
     if (st != INKLING_OK) return st;
     cudaError_t e = launch_sconv_kv(sp, stream, /*zero_hist=*/true);
     if (e != cudaSuccess) return cuda_fail(e, "attn_prefill (two-pass) sconv launch");
-    e = launch_attn_prefill_paged(pp, tm_q, tm_k, tm_v, stream, p->seq_len);
+    e = launch_attn_prefill_paged(pp, tm_q, tm_k, tm_v, stream, p->seq_len, sms);
     if (e != cudaSuccess) return cuda_fail(e, "attn_prefill (two-pass) paged launch");
     return INKLING_OK;
 }
@@ -453,9 +453,10 @@ inkling_status inkling_attn_prefill(const inkling_prefill_params *p, inkling_str
         }
         two_pass = room && two_pass_fits(p);
     }
-    inkling_status st = check_device(nullptr);
+    int sms = 0;
+    inkling_status st = check_device(&sms);
     if (st != INKLING_OK) return st;
-    if (two_pass) return prefill_two_pass(p, (cudaStream_t)stream);
+    if (two_pass) return prefill_two_pass(p, (cudaStream_t)stream, sms);
 
     const cuuint64_t T = (cuuint64_t)p->seq_len, B = (cuuint64_t)p->batch;
     const cuuint64_t Hq = (cuuint64_t)p->num_q_heads, Hkv = (cuuint64_t)p->num_kv_heads;
@@ -582,13 +583,14 @@ inkling_status inkling_attn_prefill_paged(const inkling_prefill_paged_params *p,
     if (!aligned16(p->q) || !aligned16(p->k_cache) || !aligned16(p->v_cache) || !aligned16(p->out))
         return fail(INKLING_ERR_INVALID, "q, caches and out must be 16-byte aligned");
     if (((uintptr_t)p->bias & 3u) != 0) return fail(INKLING_ERR_INVALID, "bias must be 4-byte aligned");
-    inkling_status st = check_device(nullptr);
+    int sms = 0;
+    inkling_status st = check_device(&sms);
     if (st != INKLING_OK) return st;
     CUtensorMap tm_q, tm_k, tm_v;
     if ((st = paged_maps(p->q, p->total_q, p->num_q_heads, p->k_cache, p->v_cache, p->num_blocks,
                          p->num_kv_heads, &tm_q, &tm_k, &tm_v)) != INKLING_OK)
         return st;
-    cudaError_t e = launch_attn_prefill_paged(*p, tm_q, tm_k, tm_v, (cudaStream_t)stream);
+    cudaError_t e = launch_attn_prefill_paged(*p, tm_q, tm_k, tm_v, (cudaStream_t)stream, 0, sms);
     if (e != cudaSuccess) return cuda_fail(e, "attn_prefill_paged launch");
     return INKLING_OK;
 }
