@@ -197,7 +197,7 @@ def hbm_roofline(achieved, kernel, traffic=None):
 # ----------------------------------------------------------- GPU workload --
 
 class PrefillStep:
-    """One prefill call on the automatic path (two-pass from 2048 tokens:
+    """One prefill call on the automatic path (two-pass from 2048 tokens per call:
     sconv into a preallocated workspace, then the paged prefill kernel; fused
     below), plus the fused kernel and the cache-filling variants of the same
     call, and the two passes as separate public calls for their timings."""

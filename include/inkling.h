@@ -174,17 +174,19 @@ inkling_status inkling_sconv_kv(const inkling_sconv_params *p, inkling_stream_t 
  *    num_blocks*Hkv*128 < 2^31 and B*T*Hq < 2^31 (the workspace blocks
  *    count when there is no cache); without a cache, workspace_bytes must be
  *    at least inkling_attn_prefill_workspace_bytes(p).
- *  - INKLING_PREFILL_AUTO: the two-pass path when T >= INKLING_PREFILL_TWO_PASS_MIN_T
- *    and it is possible (a cache, or a large enough workspace, and the size
- *    limits above), else the fused one.  On B200 the two-pass path is 9-12%
- *    faster from 2048 tokens up (the conversion is done once per token rather
- *    than once per covering block, for ~1.6% extra HBM traffic), and the
- *    fused one is faster below ~1024 tokens (one launch instead of two).
+ *  - INKLING_PREFILL_AUTO: the two-pass path when B*T >= INKLING_PREFILL_TWO_PASS_MIN_TOKENS
+ *    and T >= INKLING_PREFILL_TWO_PASS_MIN_T, and it is possible (a cache, or a
+ *    large enough workspace, and the size limits above), else the fused one.
+ *    On B200 the two-pass path is 9-23% faster there (the conversion is done
+ *    once per token rather than once per covering block, for ~1.6% extra HBM
+ *    traffic), and the fused one is faster on smaller calls (one launch
+ *    instead of two, and its CTA pairs share each tile).
  * -------------------------------------------------------------------------- */
 #define INKLING_PREFILL_AUTO 0
 #define INKLING_PREFILL_FUSED 1
 #define INKLING_PREFILL_TWO_PASS 2
-#define INKLING_PREFILL_TWO_PASS_MIN_T 2048
+#define INKLING_PREFILL_TWO_PASS_MIN_TOKENS 2048
+#define INKLING_PREFILL_TWO_PASS_MIN_T 512
 
 typedef struct {
     const void *q;        /* device [B, T, Hq, d] bf16 */
@@ -221,10 +223,10 @@ inkling_status inkling_attn_prefill(const inkling_prefill_params *p, inkling_str
 
 /* Bytes of workspace inkling_attn_prefill(p) uses: 2 * B * ceil(T/128) * Hkv
  * * 128 * 128 * 2 (post-sconv keys and values in the paged layout) when p's
- * path is TWO_PASS, or AUTO and T >= INKLING_PREFILL_TWO_PASS_MIN_T, with no
- * cache given; 0 when the call needs none (the fused path, a cache given, B
- * or T zero) or p is NULL.  Only the sizes, path and cache pointer of p are
- * read. */
+ * path is TWO_PASS, or AUTO with B*T >= INKLING_PREFILL_TWO_PASS_MIN_TOKENS
+ * and T >= INKLING_PREFILL_TWO_PASS_MIN_T, with no cache given; 0 when the
+ * call needs none (the fused path, a cache given, B or T zero) or p is NULL.
+ * Only the sizes, path and cache pointer of p are read. */
 size_t inkling_attn_prefill_workspace_bytes(const inkling_prefill_params *p);
 
 /* --------------------------------------------------------------------------

@@ -21,7 +21,8 @@ INKLING_OK, INKLING_ERR_INVALID, INKLING_ERR_UNSUPPORTED, INKLING_ERR_CUDA = 0, 
 STATUS_TIMEOUT, STATUS_BAD_BLOCK, STATUS_BAD_LENGTH = 1, 2, 4
 HEAD_DIM = 128
 BLOCK_SIZE = 128
-INKLING_PREFILL_TWO_PASS_MIN_T = 2048
+INKLING_PREFILL_TWO_PASS_MIN_TOKENS = 2048
+INKLING_PREFILL_TWO_PASS_MIN_T = 512
 
 EXPORTED = (
     "inkling_last_error",

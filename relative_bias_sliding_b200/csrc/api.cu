@@ -281,7 +281,8 @@ bool two_pass_fits(const inkling_prefill_params *p) {
 
 bool wants_two_pass(const inkling_prefill_params *p) {
     return p->path == INKLING_PREFILL_TWO_PASS ||
-           (p->path == INKLING_PREFILL_AUTO && p->seq_len >= INKLING_PREFILL_TWO_PASS_MIN_T);
+           (p->path == INKLING_PREFILL_AUTO && p->seq_len >= INKLING_PREFILL_TWO_PASS_MIN_T &&
+            (long)p->batch * p->seq_len >= INKLING_PREFILL_TWO_PASS_MIN_TOKENS);
 }
 
 // Pass 1: the sconv of all T raw keys/values of every sequence, zero history,

@@ -62,6 +62,7 @@ int main(void) {{
   F(inkling_sconv_out_sharded_params, channels)
   printf("paths %d%d%d\\n", INKLING_PREFILL_AUTO, INKLING_PREFILL_FUSED, INKLING_PREFILL_TWO_PASS);
   printf("min_t %d\\n", INKLING_PREFILL_TWO_PASS_MIN_T);
+  printf("min_tokens %d\\n", INKLING_PREFILL_TWO_PASS_MIN_TOKENS);
   return 0;
 }}""")
     exe = tmp_path / "sizes"
@@ -90,6 +91,7 @@ int main(void) {{
     P = binding.PREFILL_PATHS
     assert out["paths"] == f"{P['auto']}{P['fused']}{P['two_pass']}"
     assert int(out["min_t"]) == binding.INKLING_PREFILL_TWO_PASS_MIN_T
+    assert int(out["min_tokens"]) == binding.INKLING_PREFILL_TWO_PASS_MIN_TOKENS
     H = binding.SconvOutShardedParams
     assert int(out["sharded"]) == ctypes.sizeof(H)
     for m in ("state", "n_ranks", "channels"):
@@ -128,17 +130,22 @@ def test_workspace_bytes(lib):
 def test_prefill_workspace_bytes(lib):
     """The two-pass prefill's scratch: post-sconv K and V of ceil(T/128) blocks
     per sequence; none for the fused path, with a cache, or below the
-    automatic path's length threshold."""
+    automatic path's thresholds (B*T >= 2048 tokens and T >= 512)."""
     f = lib.inkling_attn_prefill_workspace_bytes
     p = binding.PrefillParams()
     p.batch, p.seq_len, p.num_q_heads, p.num_kv_heads, p.head_dim = 4, 8192, 64, 8, 128
     assert f(ctypes.byref(p)) == 2 * 4 * 64 * 8 * 128 * 128 * 2  # auto, 8192 tokens
     p.path = binding.PREFILL_PATHS["fused"]
     assert f(ctypes.byref(p)) == 0
-    p.path, p.seq_len = binding.PREFILL_PATHS["auto"], 2047
-    assert f(ctypes.byref(p)) == 0  # below the threshold the automatic path fuses
+    p.path, p.seq_len = binding.PREFILL_PATHS["auto"], 511
+    assert f(ctypes.byref(p)) == 0  # T below 512: the automatic path fuses
+    p.seq_len = 512
+    assert f(ctypes.byref(p)) == 2 * 4 * 4 * 8 * 128 * 128 * 2  # B*T = 2048
+    p.batch, p.seq_len = 1, 2047
+    assert f(ctypes.byref(p)) == 0  # B*T below 2048
     p.seq_len = 2048
-    assert f(ctypes.byref(p)) == 2 * 4 * 16 * 8 * 128 * 128 * 2
+    assert f(ctypes.byref(p)) == 2 * 1 * 16 * 8 * 128 * 128 * 2
+    p.batch = 4
     p.path, p.seq_len, p.batch = binding.PREFILL_PATHS["two_pass"], 300, 3  # ragged: 3 blocks
     assert f(ctypes.byref(p)) == 2 * 3 * 3 * 8 * 128 * 128 * 2
     p.k_cache = ctypes.c_void_p(1 << 20)
@@ -146,7 +153,8 @@ def test_prefill_workspace_bytes(lib):
     p.k_cache, p.seq_len = None, 0
     assert f(ctypes.byref(p)) == 0
     assert f(None) == 0
-    assert binding.INKLING_PREFILL_TWO_PASS_MIN_T == 2048
+    assert binding.INKLING_PREFILL_TWO_PASS_MIN_T == 512
+    assert binding.INKLING_PREFILL_TWO_PASS_MIN_TOKENS == 2048
 
 
 def test_prefill_path_validation_rejects_before_launch(lib):

@@ -111,27 +111,28 @@ def test_prefill_window_at_least_T_equals_full(path):
     assert torch.equal(full, win)
 
 
-@pytest.mark.parametrize("T", [2047, 2048])
-def test_prefill_auto_path_follows_the_length_threshold(T):
-    """The automatic path fuses below 2048 tokens and runs the two passes from
-    there: the library asks for a workspace only from 2048 tokens, and a
-    workspace passed then is written by the first pass.  The two paths give the
-    same bits: the same MMA order and softmax code over the same post-sconv
-    keys and values."""
+@pytest.mark.parametrize("B,T,two", [(1, 2047, False), (1, 2048, True), (4, 511, False),
+                                     (4, 512, True), (2, 1000, False)])
+def test_prefill_auto_path_follows_the_thresholds(B, T, two):
+    """The automatic path runs the two passes when B*T >= 2048 tokens and
+    T >= 512, and fuses otherwise: the library asks for a workspace only then,
+    and a workspace passed then is written by the first pass.  The two paths
+    give the same bits: the same MMA order and softmax code over the same
+    post-sconv keys and values."""
     need_gpu()
     Hq, Hkv = 16, 2
-    spec = scaled(WORKLOADS["prefill_swa_b4_t8192"], B=1, T=T, Hq=Hq, Hkv=Hkv, window=1000,
-                  D_max=3000, seed=T)
+    spec = scaled(WORKLOADS["prefill_swa_b4_t8192"], B=B, T=T, Hq=Hq, Hkv=Hkv, window=1000,
+                  D_max=3000, seed=T + B)
     t = make_prefill(spec)
     dev = {k: v.cuda() for k, v in t.items()}
-    need = ink.prefill_workspace_bytes(1, T, Hq, Hkv)
-    assert (need > 0) == (T >= 2048)
+    need = ink.prefill_workspace_bytes(B, T, Hq, Hkv)
+    assert (need > 0) == two
     ws = torch.full((max(need, 16),), 0xff, dtype=torch.uint8, device="cuda")
-    lse = torch.empty((1, Hq, T), dtype=torch.float32, device="cuda")
+    lse = torch.empty((B, Hq, T), dtype=torch.float32, device="cuda")
     auto = ink.attn_prefill(dev["q"], dev["k_raw"], dev["v_raw"], dev["w_k"], dev["w_v"],
                             dev["bias"], window=1000, lse=lse, workspace=ws)
     torch.cuda.synchronize()
-    assert bool((ws != 0xff).any()) == (T >= 2048)
+    assert bool((ws != 0xff).any()) == two
     for path in PATHS:
         out, lse2 = _run(t, 1000, path=path)
         assert torch.equal(auto.view(torch.int16), out.view(torch.int16)), path
