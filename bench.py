@@ -57,6 +57,8 @@ MEASURED_TRAFFIC = {
     # the pair kernel on the fused one (" fused")
     "prefill_swa_b4_t8192": 676_789_248 + 496_522_240,
     "prefill_swa_b4_t8192 fused": 680_339_712 + 501_876_992,
+    "prefill_paged_swa_b4_t8192": 677_420_032 + 495_994_368,
+    "prefill_chunked_swa_b4_c2048": 238_170_880 + 99_981_312,
     "decode_swa_s64": 1_080_809_216 + 3_773_440,
     "decode_mtp9_swa_s64": 1_089_955_584 + 8_819_968,
 }
