@@ -191,7 +191,10 @@ attn_prefill_paged_kernel(const __grid_constant__ CUtensorMap tm_q,
 
     if (warp < 8) {
         // ================================================== softmax (2 WGs) ==
-        setmaxnreg_inc184();
+        if constexpr (kPersist)
+            setmaxnreg_inc192();
+        else
+            setmaxnreg_inc200();
         const int t = warp >> 2;
         int k_base = 0;        // key tiles this group has processed (S_FULL, bias parities)
         uint32_t items = 0;    // items this group has finished (O_DONE parity)
@@ -222,7 +225,10 @@ attn_prefill_paged_kernel(const __grid_constant__ CUtensorMap tm_q,
     } else if (warp < 12) {
         setmaxnreg_dec24();
     } else {
-        setmaxnreg_dec120();
+        if constexpr (kPersist)
+            setmaxnreg_dec104();
+        else
+            setmaxnreg_dec88();
         if (warp == 12 && lane == 0) {
             // ============================================== TMA producer ==
             tma_prefetch_desc(&tm_q);

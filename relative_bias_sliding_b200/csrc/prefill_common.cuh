@@ -82,12 +82,15 @@ INK_DEV void setmaxnreg_dec64() { asm volatile("setmaxnreg.dec.sync.aligned.u32 
 // plain prefill keeps its split: 696 against 689).
 INK_DEV void setmaxnreg_inc168() { asm volatile("setmaxnreg.inc.sync.aligned.u32 168;"); }
 INK_DEV void setmaxnreg_dec96() { asm volatile("setmaxnreg.dec.sync.aligned.u32 96;"); }
-// The split of the paged prefill, which has no sconv warps: its four idle
-// warps keep the minimum and the producer / MMA group gets 120, for the
-// walk over work items (8 x 184 + 4 x 24 + 4 x 120 = 2048 = 16 warps x 128,
-// the launch's registers).
+// The splits of the paged prefill, which has no sconv warps: its four idle
+// warps keep the minimum, and the softmax groups take most of the rest.
+// Persistent walk: 8 x 192 + 4 x 24 + 4 x 104 = 2048; one item per CTA:
+// 8 x 200 + 4 x 24 + 4 x 88 = 2048 (16 warps x 128, the launch's registers).
+INK_DEV void setmaxnreg_inc192() { asm volatile("setmaxnreg.inc.sync.aligned.u32 192;"); }
+INK_DEV void setmaxnreg_inc200() { asm volatile("setmaxnreg.inc.sync.aligned.u32 200;"); }
 INK_DEV void setmaxnreg_dec24() { asm volatile("setmaxnreg.dec.sync.aligned.u32 24;"); }
-INK_DEV void setmaxnreg_dec120() { asm volatile("setmaxnreg.dec.sync.aligned.u32 120;"); }
+INK_DEV void setmaxnreg_dec104() { asm volatile("setmaxnreg.dec.sync.aligned.u32 104;"); }
+INK_DEV void setmaxnreg_dec88() { asm volatile("setmaxnreg.dec.sync.aligned.u32 88;"); }
 
 // Taps of 8 consecutive channels starting at `wg` ([C, 4] fp32), as channel
 // pairs: w[tap][p] = (w[2p][tap], w[2p+1][tap]).
