@@ -55,10 +55,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 MEASURED_TRAFFIC = {
     # the prefill call's dominant kernel: the paged kernel on the two-pass path,
     # the pair kernel on the fused one (" fused")
-    "prefill_swa_b4_t8192": 676_789_248 + 496_522_240,
+    "prefill_swa_b4_t8192": 676_627_968 + 496_061_952,
     "prefill_swa_b4_t8192 fused": 680_339_712 + 501_876_992,
-    "prefill_paged_swa_b4_t8192": 677_420_032 + 495_994_368,
-    "prefill_chunked_swa_b4_c2048": 238_170_880 + 99_981_312,
+    "prefill_paged_swa_b4_t8192": 676_296_960 + 498_352_896,
+    "prefill_chunked_swa_b4_c2048": 237_998_336 + 99_810_560,
     "decode_swa_s64": 1_080_809_216 + 3_773_440,
     "decode_mtp9_swa_s64": 1_089_955_584 + 8_819_968,
 }
