@@ -260,7 +260,10 @@ INK_DEV void softmax_role(const PrefillArgs &a, float *bias_sm, uint64_t *s_full
     const int W = a.window, Dm = a.d_max, T = key_end;
     float m_ref = -INFINITY, l = 0.f;
     const int o_rd = 127 - u, sh = o_rd & 3;  // this row's start in the staged diagonal
-    bool dead = false;
+    // an item started after an abort waits on nothing: its barriers may be
+    // phases behind, where a parity test could pass on an older phase; its
+    // rows are written as NaN (warp-uniform, for the warp-wide TMEM loads)
+    bool dead = __any_sync(0xffffffffu, *abort_flag != 0);
     int k = 0;
     for (int n = lo; n <= hi; ++n, ++k) {
         const int j0 = n * 128;
