@@ -698,14 +698,27 @@ def run_reference(args):
             vals.append(v)
             descs.append(desc)
     value = statistics.mean(vals)
+    # the same config as this bench's own arm: the default step is the
+    # sliding-window prefill plus the sliding-window decode step
+    workload = name if args.workload else f"{DEFAULT_PREFILL} + {DEFAULT_DECODE}"
+    config = {"workload": workload, "parallelism": f"replica per GPU x{args.gpus}",
+              "l2": "not applicable: the oracle runs on the host cores"}
+    if isinstance(spec, PrefillSpec):
+        config["prefill_path"] = "not applicable: the oracle computes every row directly"
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": unit,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": name},
+            "data": "synthetic", "config": config,
             "cpu_baseline": {"value": value, "unit": unit, "cores": thr, "kind": "oracle",
                              "sample": descs[0]},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
+    if not args.workload:
+        # the decode half of the default step, as in this bench's own line
+        dv, ddesc, dthr = oracle_decode_sample(WORKLOADS[DEFAULT_DECODE], per_step / 2)
+        line["decode"] = {"workload": DEFAULT_DECODE, "value": dv, "unit": "GB/s",
+                          "cpu_baseline": {"value": dv, "unit": "GB/s", "cores": dthr,
+                                           "kind": "oracle", "sample": ddesc}}
     print(json.dumps(line), flush=True)
     return 0
 
